@@ -1,0 +1,322 @@
+/*
+ * Scalar CPU oracle for per-token-group activation quantization.
+ *
+ * TEST INFRASTRUCTURE ONLY.  This is the plain, slow, obviously correct
+ * statement of what the quantization path computes.  Only the test suite, the
+ * smoke check and the benchmark's CPU-baseline leg load it.  It shares no code,
+ * header, table or constant generator with the CUDA library, and the product
+ * path never calls it.
+ *
+ * What it follows (page title, section):
+ *   [PR]  sglang PR #30924 report, "[JIT] Trait-driven per_token_group_quant:
+ *         unify the quant kernel family (flat + masked)":
+ *           - 实现拆解 item 1: the variant axes (input/output dtype, group size,
+ *             fp32 or UE8M0 scale, row- or column-major scale layout, fused
+ *             silu_and_mul, flat or masked dispatch);
+ *           - 实现拆解 item 2: masked dispatch driven by masked_m / expected_m;
+ *           - 关键源码片段, ref_fp8_ue8m0: group absmax floored at EPS,
+ *             raw = amax / FMAX with FMAX = 448, UE8M0 exponent = biased exponent
+ *             of raw plus one when raw's mantissa is nonzero, codes from a
+ *             saturating quantize clamped to [-FMAX, FMAX];
+ *           - _jit_module snippet: the `aligned` flag (group count a multiple
+ *             of 4, UE8M0 only) and the scale layout flags;
+ *           - 关键文件 / 风险与影响: the INT8 path (ref_int8) with identical
+ *             scales, i.e. scale = amax / 127.
+ *   [TF]  "tf-kernel 安装与使用" (TeleFuser), 使用示例: silu_and_mul splits the
+ *         last dimension into two halves of equal width.
+ *   [FI]  "FlashInfer GEMM 学习笔记", sections 6-7: block-scaled consumers want
+ *         TMA-aligned packed scales; grouped-masked GEMMs take a fixed
+ *         expected_m plus a per-expert masked_m.
+ *
+ * Readings taken where the pages are silent (each one is listed with its
+ * reason in the design notes):
+ *   - EPS = 1e-10f (the snippet names EPS without printing its value).
+ *   - gate is the first half of a fused row, up the second half.
+ *   - the SiLU-and-mul product is formed in double and rounded once to fp32;
+ *     it is never rounded to the input dtype.
+ *   - every rounding is to nearest, ties to even; E4M3 is the OCP "fn"
+ *     variant (no infinities, 448 largest finite), zero keeps the sign of t.
+ *   - column-major layouts pad the row count to a multiple of 4 (16 bytes of
+ *     fp32 or one int32 word per 4 rows), padding rows are never written.
+ *   - the UE8M0-packed layout stores the exponents of groups 4j..4j+3 of a
+ *     row in one little-endian int32 word; bytes for groups past the last one
+ *     are 0.
+ *
+ * Build: gcc -O2 -std=c11 -fPIC -shared -ffp-contract=off (no fast-math).
+ * Floating point: C float arithmetic is IEEE binary32 with round-to-nearest
+ * (FLT_EVAL_METHOD 0 on x86-64 and aarch64); fp-contract is off so no
+ * multiply-add is fused behind the reader's back.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* ---- constants of the method (values, not code, shared with nobody) ---- */
+#define PQGO_FMAX_E4M3 448.0f   /* largest finite E4M3 value ([PR] FMAX)       */
+#define PQGO_FMAX_INT8 127.0f   /* INT8 scale divisor ([PR] ref_int8)          */
+#define PQGO_EPS 1e-10f         /* absmax floor ([PR] "不低于 EPS")             */
+
+/* layouts understood by the oracle (numbered for the Python wrapper) */
+enum { PQGO_ROW = 0, PQGO_COL = 1, PQGO_PACKED = 2 };
+
+/* ------------------------------------------------------------------------ */
+/* Input decoding                                                            */
+/* ------------------------------------------------------------------------ */
+
+/* bfloat16 is the upper 16 bits of an IEEE binary32 (1 sign, 8 exponent,
+ * 7 fraction bits), so widening is exact: put the bits back on top. */
+static float decode_bf16(uint16_t h) {
+    uint32_t w = (uint32_t)h << 16;
+    float f;
+    memcpy(&f, &w, sizeof f);
+    return f;
+}
+
+/* IEEE binary16: 1 sign bit, 5 exponent bits (bias 15), 10 fraction bits.
+ * Subnormals are m * 2^-24; normals are (1024 + m) * 2^(e - 25). */
+static float decode_f16(uint16_t h) {
+    int sign = (h >> 15) & 1;
+    int e = (h >> 10) & 0x1F;
+    int m = h & 0x3FF;
+    double v;
+    if (e == 0)
+        v = ldexp((double)m, -24);
+    else if (e == 31)
+        v = m ? NAN : INFINITY;
+    else
+        v = ldexp(1024.0 + (double)m, e - 25);
+    return (float)(sign ? -v : v);
+}
+
+float pqgo_decode(uint16_t bits, int in_fp16) {
+    return in_fp16 ? decode_f16(bits) : decode_bf16(bits);
+}
+
+/* ------------------------------------------------------------------------ */
+/* Fused prologue: y = silu(gate) * up, silu(g) = g / (1 + e^-g)  [PR] item 1 */
+/* ------------------------------------------------------------------------ */
+
+float pqgo_silu_mul(float gate, float up) {
+    double g = (double)gate;
+    double silu = g / (1.0 + exp(-g));
+    return (float)(silu * (double)up);
+}
+
+/* ------------------------------------------------------------------------ */
+/* Group statistics and scales                                               */
+/* ------------------------------------------------------------------------ */
+
+/* absmax of one group, floored at EPS  ([PR] 关键源码片段, _group_amax) */
+float pqgo_group_amax(const float *v, int64_t n) {
+    float a = 0.0f;
+    for (int64_t i = 0; i < n; ++i) {
+        float m = fabsf(v[i]);
+        if (m > a) a = m;
+    }
+    if (a < PQGO_EPS) a = PQGO_EPS;
+    return a;
+}
+
+/* fp32 scale: amax / 448 for E4M3, amax / 127 for INT8, one IEEE division. */
+float pqgo_scale_fp32(float amax, int out_int8) {
+    return out_int8 ? amax / PQGO_FMAX_INT8 : amax / PQGO_FMAX_E4M3;
+}
+
+/* UE8M0 exponent byte, the pages' steps in their order ([PR] ref_fp8_ue8m0):
+ * raw = amax / FMAX in fp32; take raw's biased exponent field; add one when
+ * raw's 23-bit mantissa is nonzero (rounds the scale up to a power of two).
+ * The scale is 2^(byte - 127). */
+int pqgo_ue8m0_exponent(float amax) {
+    float raw = amax / PQGO_FMAX_E4M3;
+    uint32_t bits;
+    memcpy(&bits, &raw, sizeof bits);
+    int biased = (int)((bits >> 23) & 0xFF);
+    int bump = (bits & 0x7FFFFF) != 0;
+    return biased + bump;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Output encoders                                                           */
+/* ------------------------------------------------------------------------ */
+
+/* Saturating cast to OCP FP8 E4M3 ("fn": no infinities, S.1111.111 is NaN).
+ * Codes: sign bit, 4 exponent bits (bias 7), 3 mantissa bits.  Normal values
+ * are (1 + m/8) * 2^(e - 7) for e = 1..15 (m <= 6 at e = 15, so 448 is the
+ * largest finite value); subnormals are (m/8) * 2^-6.  The value is first
+ * clamped to [-448, 448] ([PR] _quantize(..., -FMAX, FMAX)), then rounded to
+ * the nearest representable magnitude with ties to an even mantissa.  A value
+ * that rounds to zero keeps the sign of t. */
+uint8_t pqgo_e4m3_encode(float t) {
+    uint8_t sign = signbit(t) ? 0x80 : 0x00;
+    double a = fabs((double)t);
+    if (a > 448.0) a = 448.0;
+    /* spacing of the representable values that bracket a */
+    int E = (a >= ldexp(1.0, -6)) ? ilogb(a) : -6;
+    double quantum = ldexp(1.0, E - 3);
+    double n = nearbyint(a / quantum); /* exact quotient; ties to even */
+    double r = n * quantum;            /* may carry into the next binade */
+    if (r == 0.0) return sign;
+    int Er = ilogb(r);
+    if (Er < -6) /* subnormal: r = m * 2^-9, m in 1..7 */
+        return (uint8_t)(sign | (uint8_t)(r / ldexp(1.0, -9)));
+    {
+        int exp_field = Er + 7;
+        int mant = (int)(r / ldexp(1.0, Er - 3)) - 8;
+        return (uint8_t)(sign | (exp_field << 3) | mant);
+    }
+}
+
+/* Saturating cast to INT8: round to nearest integer, ties to even, then
+ * clamp to [-128, 127]. */
+int8_t pqgo_int8_encode(float t) {
+    double n = nearbyint((double)t);
+    if (n > 127.0) n = 127.0;
+    if (n < -128.0) n = -128.0;
+    return (int8_t)n;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Scale layouts                                                             */
+/* ------------------------------------------------------------------------ */
+
+/* rows of one expert's column-major scale plane: M rounded up to 4 */
+static int64_t padded_rows(int64_t M) { return (M + 3) / 4 * 4; }
+
+/* Size in bytes of the scale buffer for E experts of M rows of K outputs. */
+int64_t pqgo_scales_nbytes(int64_t E, int64_t M, int64_t K, int G,
+                           int scale_ue8m0, int layout) {
+    int64_t ng = K / G;
+    int64_t elem = scale_ue8m0 ? 1 : 4;
+    if (layout == PQGO_ROW) return E * M * ng * elem;
+    if (layout == PQGO_COL) return E * ng * padded_rows(M) * elem;
+    /* packed: int32 words, ceil(ng / 4) per row */
+    return E * ((ng + 3) / 4) * padded_rows(M) * 4;
+}
+
+/* ------------------------------------------------------------------------ */
+/* The whole quantization                                                    */
+/* ------------------------------------------------------------------------ */
+
+/* Quantize E experts of M rows (E = 1, masked_m = NULL: flat dispatch).
+ *   in      : [E][M][K] (or [E][M][2K] when fused: gate | up), raw 16-bit
+ *             bf16 or fp16 patterns
+ *   out     : [E][M][K] one code byte per element
+ *   scales  : layout-dependent (see pqgo_scales_nbytes)
+ *   masked_m: host array of E row counts, or NULL.  Rows m >= masked_m[e]
+ *             (clamped to [0, M]) are not touched; neither are padding rows.
+ * Returns 0, -1 for an invalid argument, -2 for a non-finite input value. */
+int pqgo_quant(const uint16_t *in, uint8_t *out, void *scales, int64_t E,
+               int64_t M, int64_t K, int G, int in_fp16, int out_int8,
+               int scale_ue8m0, int layout, int fused,
+               const int32_t *masked_m) {
+    if (E < 1 || M < 0 || K <= 0 || G <= 0 || K % G != 0) return -1;
+    if (layout < PQGO_ROW || layout > PQGO_PACKED) return -1;
+    if (scale_ue8m0 && out_int8) return -1;       /* UE8M0 pairs with FMAX */
+    if (layout == PQGO_PACKED && !scale_ue8m0) return -1;
+    if (masked_m && layout != PQGO_ROW && M % 4 != 0) return -1;
+
+    const int64_t ng = K / G;
+    const int64_t in_width = fused ? 2 * K : K;
+    const int64_t mpad = padded_rows(M);
+    float *v = (float *)malloc(sizeof(float) * (size_t)G);
+    if (!v) return -1;
+    int status = 0;
+
+    for (int64_t e = 0; e < E && status == 0; ++e) {
+        int64_t rows = M;
+        if (masked_m) {
+            rows = masked_m[e];
+            if (rows < 0) rows = 0;
+            if (rows > M) rows = M;
+        }
+        for (int64_t m = 0; m < rows && status == 0; ++m) {
+            const uint16_t *xrow = in + (e * M + m) * in_width;
+            uint8_t *qrow = out + (e * M + m) * K;
+            for (int64_t g = 0; g < ng; ++g) {
+                /* 1. decode (and fuse) the G values of this group */
+                for (int i = 0; i < G; ++i) {
+                    float x = pqgo_decode(xrow[g * G + i], in_fp16);
+                    if (fused) {
+                        float up = pqgo_decode(xrow[K + g * G + i], in_fp16);
+                        if (!isfinite(x) || !isfinite(up)) { status = -2; break; }
+                        x = pqgo_silu_mul(x, up);
+                    }
+                    if (!isfinite(x)) { status = -2; break; }
+                    v[i] = x;
+                }
+                if (status) break;
+
+                /* 2. absmax and 3. scale */
+                float amax = pqgo_group_amax(v, G);
+                float s;
+                int ebyte = 0;
+                if (scale_ue8m0) {
+                    ebyte = pqgo_ue8m0_exponent(amax);
+                    s = ldexpf(1.0f, ebyte - 127);
+                } else {
+                    s = pqgo_scale_fp32(amax, out_int8);
+                }
+
+                /* 4. codes: saturating cast of x / s */
+                for (int i = 0; i < G; ++i) {
+                    float t = v[i] / s;
+                    qrow[g * G + i] = out_int8 ? (uint8_t)pqgo_int8_encode(t)
+                                               : pqgo_e4m3_encode(t);
+                }
+
+                /* 5. scale store */
+                if (layout == PQGO_ROW) {
+                    int64_t idx = (e * M + m) * ng + g;
+                    if (scale_ue8m0) ((uint8_t *)scales)[idx] = (uint8_t)ebyte;
+                    else ((float *)scales)[idx] = s;
+                } else if (layout == PQGO_COL) {
+                    int64_t idx = e * ng * mpad + g * mpad + m;
+                    if (scale_ue8m0) ((uint8_t *)scales)[idx] = (uint8_t)ebyte;
+                    else ((float *)scales)[idx] = s;
+                } else {
+                    int64_t nwords = (ng + 3) / 4;
+                    int64_t word = e * nwords * mpad + (g / 4) * mpad + m;
+                    ((uint8_t *)scales)[word * 4 + (g % 4)] = (uint8_t)ebyte;
+                }
+            }
+            /* packed words: exponent bytes of groups past the last are 0 */
+            if (status == 0 && layout == PQGO_PACKED && ng % 4 != 0) {
+                int64_t nwords = (ng + 3) / 4;
+                int64_t word = e * nwords * mpad + (ng / 4) * mpad + m;
+                for (int64_t b = ng % 4; b < 4; ++b)
+                    ((uint8_t *)scales)[word * 4 + b] = 0;
+            }
+        }
+    }
+    free(v);
+    return status;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Array forms of the element functions, for the pin tests                   */
+/* ------------------------------------------------------------------------ */
+
+void pqgo_decode_n(const uint16_t *bits, float *out, int64_t n, int in_fp16) {
+    for (int64_t i = 0; i < n; ++i) out[i] = pqgo_decode(bits[i], in_fp16);
+}
+
+void pqgo_silu_mul_n(const float *gate, const float *up, float *y, int64_t n) {
+    for (int64_t i = 0; i < n; ++i) y[i] = pqgo_silu_mul(gate[i], up[i]);
+}
+
+void pqgo_e4m3_encode_n(const float *t, uint8_t *q, int64_t n) {
+    for (int64_t i = 0; i < n; ++i) q[i] = pqgo_e4m3_encode(t[i]);
+}
+
+void pqgo_int8_encode_n(const float *t, int8_t *q, int64_t n) {
+    for (int64_t i = 0; i < n; ++i) q[i] = pqgo_int8_encode(t[i]);
+}
+
+void pqgo_ue8m0_exponent_n(const float *amax, uint8_t *e, int64_t n) {
+    for (int64_t i = 0; i < n; ++i) e[i] = (uint8_t)pqgo_ue8m0_exponent(amax[i]);
+}
+
+void pqgo_scale_fp32_n(const float *amax, float *s, int64_t n, int out_int8) {
+    for (int64_t i = 0; i < n; ++i) s[i] = pqgo_scale_fp32(amax[i], out_int8);
+}

@@ -1,0 +1,459 @@
+"""Pins of the CPU oracle to facts that do not come from the oracle itself.
+
+Every check here compares the oracle against something independent of it:
+- values worked by hand (tests/golden/worked_groups.json, each with its citation);
+- closed forms, computed exactly in float64 integer arithmetic;
+- brute-force searches over a table built from the OCP FP8 definition;
+- library routines (torch's float8_e4m3fn cast, numpy/torch float conversions,
+  torch's float64 SiLU);
+- invariants the quantization must satisfy.
+The checks are chosen so that a dropped term, a wrong sign or index, or a
+transposed operand in the oracle fails at least one of them.  CPU only.
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from precision_activation_quantization_b200 import inputs
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "worked_groups.json")
+
+
+# --------------------------------------------------------------------------
+# Independent reference facts
+# --------------------------------------------------------------------------
+
+def e4m3_table() -> np.ndarray:
+    """float64 value of each of the 256 E4M3 codes (OCP FP8, 'fn' variant)."""
+    vals = np.empty(256, np.float64)
+    for c in range(256):
+        sign = -1.0 if c & 0x80 else 1.0
+        e, m = (c >> 3) & 0xF, c & 7
+        if e == 15 and m == 7:
+            vals[c] = np.nan
+        elif e == 0:
+            vals[c] = sign * (m / 8.0) * 2.0 ** -6
+        else:
+            vals[c] = sign * (1.0 + m / 8.0) * 2.0 ** (e - 7)
+    return vals
+
+
+TABLE = e4m3_table()
+POS_CODES = np.arange(0, 0x7F)           # 0x00 .. 0x7E: finite, non-negative
+POS_VALS = TABLE[POS_CODES]
+
+
+def brute_e4m3(t) -> np.ndarray:
+    """Nearest finite E4M3 code by exhaustive search, ties to the even mantissa.
+
+    |t| is clamped to 448 first; the sign bit is t's sign (so -0 and values that
+    round to zero from below give 0x80).
+    """
+    t = np.asarray(t, np.float64).reshape(-1)
+    out = np.empty(t.size, np.uint8)
+    for lo in range(0, t.size, 1 << 15):
+        a = np.minimum(np.abs(t[lo:lo + (1 << 15)]), 448.0)
+        d = np.abs(a[:, None] - POS_VALS[None, :])
+        is_min = d == d.min(axis=1, keepdims=True)
+        n_min = is_min.sum(axis=1)
+        assert n_min.max() <= 2
+        even = (POS_CODES % 2 == 0)[None, :]
+        pick = np.where((n_min == 1)[:, None], is_min, is_min & even)
+        assert (pick.sum(axis=1) == 1).all()
+        code = POS_CODES[pick.argmax(axis=1)].astype(np.uint8)
+        out[lo:lo + a.size] = code | (np.signbit(t[lo:lo + a.size]).astype(np.uint8) << 7)
+    return out
+
+
+def exact_ue8m0(a) -> np.ndarray:
+    """127 + (smallest integer n with 448 * 2^n >= a), exactly, in float64."""
+    a = np.asarray(a, np.float32).astype(np.float64).reshape(-1)
+    n = np.floor(np.log2(a / 448.0)).astype(np.int64) - 2
+    for _ in range(6):
+        n = np.where(448.0 * np.exp2(n.astype(np.float64)) >= a, n, n + 1)
+    # n is now an upper bound; step down while the predecessor still satisfies it
+    for _ in range(6):
+        prev_ok = 448.0 * np.exp2((n - 1).astype(np.float64)) >= a
+        n = np.where(prev_ok, n - 1, n)
+    return (n + 127).astype(np.int64)
+
+
+def all_bf16_finite() -> np.ndarray:
+    bits = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    vals = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).float().numpy()
+    return bits[np.isfinite(vals)], vals[np.isfinite(vals)]
+
+
+def log_uniform(rng, n, lo_exp, hi_exp, signed=True) -> np.ndarray:
+    mag = np.exp2(rng.uniform(lo_exp, hi_exp, n)).astype(np.float32)
+    if signed:
+        mag *= np.where(rng.random(n) < 0.5, -1, 1).astype(np.float32)
+    return mag
+
+
+# --------------------------------------------------------------------------
+# Decoding
+# --------------------------------------------------------------------------
+
+def test_decode_bf16_every_pattern_matches_torch():
+    bits = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    ref = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).float().numpy()
+    got = oracle.decode(bits, "bf16")
+    assert np.array_equal(got.view(np.uint32)[np.isfinite(ref)],
+                          ref.view(np.uint32)[np.isfinite(ref)])
+    assert np.array_equal(np.isnan(got), np.isnan(ref))
+
+
+def test_decode_fp16_every_pattern_matches_numpy():
+    bits = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    ref = bits.view(np.float16).astype(np.float32)
+    got = oracle.decode(bits, "fp16")
+    fin = np.isfinite(ref)
+    assert np.array_equal(got.view(np.uint32)[fin], ref.view(np.uint32)[fin])
+    assert np.array_equal(np.isinf(got), np.isinf(ref))
+    assert np.array_equal(np.isnan(got), np.isnan(ref))
+
+
+# --------------------------------------------------------------------------
+# E4M3 encoder (P-1, P-2)
+# --------------------------------------------------------------------------
+
+def test_e4m3_table_matches_torch_and_landmarks():
+    codes = torch.arange(256, dtype=torch.int32).to(torch.uint8)
+    lib = codes.view(torch.float8_e4m3fn).double().numpy()
+    assert np.array_equal(np.isnan(lib), np.isnan(TABLE))
+    fin = ~np.isnan(TABLE)
+    assert np.array_equal(lib[fin], TABLE[fin])
+    assert TABLE[0x7E] == 448.0 and np.isnan(TABLE[0x7F]) and np.isnan(TABLE[0xFF])
+    assert TABLE[0x01] == 2.0 ** -9 and TABLE[0x08] == 2.0 ** -6
+    assert np.nanmax(TABLE) == 448.0
+
+
+def test_e4m3_round_trip_every_finite_code():
+    fin = [c for c in range(256) if not np.isnan(TABLE[c])]
+    got = oracle.e4m3_encode(TABLE[fin].astype(np.float32))
+    assert list(got) == fin
+
+
+def test_e4m3_encoder_matches_brute_force():
+    rng = np.random.default_rng(11)
+    _, bf = all_bf16_finite()
+    bf = bf[np.abs(bf) <= 1000.0]
+    vals = np.sort(POS_VALS)
+    mids = ((vals[1:] + vals[:-1]) / 2.0).astype(np.float32)   # exact in fp32
+    mids = np.concatenate([mids, np.nextafter(mids, np.float32(np.inf)),
+                           np.nextafter(mids, np.float32(-np.inf))])
+    mids = np.concatenate([mids, -mids])
+    rand = log_uniform(rng, 200_000, -14, 9.5)
+    t = np.concatenate([bf, mids, rand, np.float32([0.0, -0.0, 448.0, -448.0, 464.0,
+                                                    465.0, 1e30, -1e30])]).astype(np.float32)
+    assert np.array_equal(oracle.e4m3_encode(t), brute_e4m3(t))
+
+
+def test_e4m3_encoder_matches_torch_cast():
+    rng = np.random.default_rng(12)
+    t = log_uniform(rng, 1_000_000, -16, 9.2)
+    ref = torch.from_numpy(np.clip(t, -448.0, 448.0)).to(torch.float8_e4m3fn)
+    assert np.array_equal(oracle.e4m3_encode(t), ref.view(torch.uint8).numpy())
+
+
+def test_int8_encoder_matches_numpy_rint():
+    rng = np.random.default_rng(13)
+    t = np.concatenate([rng.uniform(-200, 200, 500_000).astype(np.float32),
+                        (np.arange(-300, 301) / 2.0).astype(np.float32)])
+    ref = np.clip(np.rint(t.astype(np.float64)), -128, 127).astype(np.int8)
+    assert np.array_equal(oracle.int8_encode(t), ref)
+
+
+# --------------------------------------------------------------------------
+# Scales (P-8)
+# --------------------------------------------------------------------------
+
+def test_ue8m0_bit_algorithm_equals_exact_ceiling():
+    rng = np.random.default_rng(14)
+    _, bf = all_bf16_finite()
+    a_bf = bf[bf >= 1e-10]
+    # random fp32 patterns in [1e-10, 2^127]
+    lo = np.float32(1e-10).view(np.uint32)
+    hi = np.float32(2.0 ** 127).view(np.uint32)
+    a_rand = rng.integers(lo, hi, size=2_000_000, dtype=np.uint32).view(np.float32)
+    # a near 7 * 2^k, where a/448 sits next to a power of two
+    k = np.arange(-30, 120, dtype=np.float64)
+    base = (7.0 * np.exp2(k)).astype(np.float32)
+    near = [base]
+    for _ in range(4):
+        near.append(np.nextafter(near[-1], np.float32(np.inf)))
+    down = [base]
+    for _ in range(4):
+        down.append(np.nextafter(down[-1], np.float32(0)))
+    a = np.concatenate([a_bf, a_rand] + near + down).astype(np.float32)
+    assert np.array_equal(oracle.ue8m0_exponent(a).astype(np.int64), exact_ue8m0(a))
+
+
+def test_fp32_scale_is_one_ieee_division():
+    rng = np.random.default_rng(15)
+    a = log_uniform(rng, 500_000, -33, 120, signed=False)
+    assert np.array_equal(oracle.scale_fp32(a, "e4m3"), a / np.float32(448.0))
+    assert np.array_equal(oracle.scale_fp32(a, "int8"), a / np.float32(127.0))
+
+
+def test_group_amax_floor_and_sign():
+    assert oracle.group_amax(np.zeros(128, np.float32)) == np.float32(1e-10)
+    v = np.zeros(128, np.float32)
+    v[77] = -3.0
+    v[5] = 2.5
+    assert oracle.group_amax(v) == 3.0
+    v = np.full(128, 1e-12, np.float32)
+    assert oracle.group_amax(v) == np.float32(1e-10)
+
+
+# --------------------------------------------------------------------------
+# Hand-worked groups (P-4, P-5, P-6)
+# --------------------------------------------------------------------------
+
+def _golden_group(entry) -> np.ndarray:
+    v = np.zeros(128, np.float32)
+    for i, x in entry["values"].items():
+        v[int(i)] = x
+    return v
+
+
+@pytest.mark.parametrize("entry", json.load(open(GOLDEN))["groups"], ids=lambda e: e["name"])
+def test_worked_group(entry):
+    v = _golden_group(entry)
+    bits = inputs.bf16_bits(v)
+    assert np.array_equal(oracle.decode(bits).view(np.uint32), v.view(np.uint32)), \
+        "worked values must be exact bf16"
+    if "ue8m0" in entry:
+        q, s = oracle.quant(bits, M=1, K=128, group=128, scale_fmt="ue8m0", layout="row")
+        assert int(s.reshape(-1)[0]) == entry["ue8m0"]["exponent"]
+        for i, c in entry["ue8m0"]["codes"].items():
+            assert int(q.reshape(-1)[int(i)]) == c, (entry["name"], i)
+    if "fp32" in entry:
+        q, s = oracle.quant(bits, M=1, K=128, group=128, scale_fmt="fp32", layout="row")
+        if "scale" in entry["fp32"]:
+            assert float(s.reshape(-1)[0]) == entry["fp32"]["scale"]
+        for i, c in entry["fp32"]["codes"].items():
+            assert int(q.reshape(-1)[int(i)]) == c, (entry["name"], i)
+    if "int8" in entry:
+        q, s = oracle.quant(bits, M=1, K=128, group=128, out_dtype="int8")
+        assert float(s.reshape(-1)[0]) == entry["int8"]["scale"]
+        for i, c in entry["int8"]["codes"].items():
+            assert int(q.view(np.int8).reshape(-1)[int(i)]) == c, (entry["name"], i)
+
+
+# --------------------------------------------------------------------------
+# Exhaustive bf16 sweep in a carrier group (P-3)
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("carrier", [448.0, 448.0 * 2 ** -20, 448.0 * 2 ** 20, 1.0,
+                                     3.140625, 1e-10])
+def test_every_bf16_value_in_a_carrier_group(carrier):
+    bits, vals = all_bf16_finite()
+    n = bits.size
+    # the carrier as the bf16 value it becomes
+    A = float(torch.tensor([carrier]).to(torch.bfloat16).float()[0])
+    x = np.full((n, 128), A, np.float32)
+    x[:, 0] = vals
+    xb = inputs.bf16_bits(x)
+    amax = np.maximum(np.maximum(np.abs(vals), np.float32(A)), np.float32(1e-10))
+
+    q, s = oracle.quant(xb, M=n, K=128, group=128, scale_fmt="ue8m0", layout="row")
+    e = exact_ue8m0(amax)
+    assert np.array_equal(s.reshape(-1).astype(np.int64), e)
+    scale = np.exp2((e - 127).astype(np.float64))
+    q = q.reshape(n, 128)
+    assert np.array_equal(q[:, 0], brute_e4m3(vals.astype(np.float64) / scale))
+    assert np.array_equal(q[:, 1], brute_e4m3(np.float64(A) / scale))
+
+    q, s = oracle.quant(xb, M=n, K=128, group=128, scale_fmt="fp32", layout="row")
+    sf = amax / np.float32(448.0)
+    assert np.array_equal(s.reshape(-1), sf)
+    q = q.reshape(n, 128)
+    assert np.array_equal(q[:, 0], brute_e4m3(vals / sf))
+    assert np.array_equal(q[:, 1], brute_e4m3(np.float32(A) / sf))
+
+    q, s = oracle.quant(xb, M=n, K=128, group=128, out_dtype="int8", layout="row")
+    si = amax / np.float32(127.0)
+    assert np.array_equal(s.reshape(-1), si)
+    ref = np.clip(np.rint((vals / si).astype(np.float64)), -128, 127).astype(np.int8)
+    assert np.array_equal(q.view(np.int8).reshape(n, 128)[:, 0], ref)
+
+
+# --------------------------------------------------------------------------
+# Invariant (P-7) and the whole path against library primitives
+# --------------------------------------------------------------------------
+
+def _f32(bits, in_dtype="bf16"):
+    return oracle.decode(bits, in_dtype)
+
+
+@pytest.mark.parametrize("scale_fmt", ["fp32", "ue8m0"])
+def test_dequant_error_bound(scale_fmt):
+    w = inputs.flat_hidden(M=256, K=7168)
+    q, s = oracle.quant(w.x, M=w.M, K=w.K, group=128, scale_fmt=scale_fmt, layout="row")
+    x = _f32(w.x).reshape(w.M, w.K // 128, 128).astype(np.float64)
+    if scale_fmt == "ue8m0":
+        sc = np.exp2(s.reshape(w.M, -1, 1).astype(np.float64) - 127)
+    else:
+        sc = s.reshape(w.M, -1, 1).astype(np.float64)
+    deq = TABLE[q.reshape(w.M, -1, 128)] * sc
+    err = np.abs(deq - x)
+    t = np.abs(x) / sc
+    normal = t >= 2.0 ** -6
+    assert (err[normal] <= 2.0 ** -4 * np.abs(x[normal]) * (1 + 2.0 ** -20)).all()
+    assert (err[~normal] <= 2.0 ** -10 * np.broadcast_to(sc, x.shape)[~normal]
+            * (1 + 2.0 ** -20)).all()
+
+
+def test_int8_dequant_error_bound():
+    w = inputs.sweep(M=512, K=4096, out_dtype="int8", group=64)
+    q, s = oracle.quant(w.x, M=w.M, K=w.K, group=64, out_dtype="int8")
+    x = _f32(w.x).reshape(w.M, -1, 64).astype(np.float64)
+    sc = s.reshape(w.M, -1, 1).astype(np.float64)
+    err = np.abs(q.view(np.int8).reshape(w.M, -1, 64) * sc - x)
+    # half a code step, plus the fp32 rounding of t = x/s (half an ulp of |t| < 128)
+    assert (err <= sc * (0.5 + 2.0 ** -18)).all()
+    assert q.view(np.int8).max() == 127 or q.view(np.int8).min() == -127
+
+
+@pytest.mark.parametrize("in_dtype,group", [("bf16", 128), ("fp16", 64), ("bf16", 32)])
+def test_whole_path_matches_torch_composition(in_dtype, group):
+    """fp32-scale E4M3 path against torch primitives (amax, fp32 division, fp8 cast)."""
+    w = inputs.sweep(M=64, K=1024, in_dtype=in_dtype, group=group)
+    q, s = oracle.quant(w.x, M=w.M, K=w.K, group=group, in_dtype=in_dtype)
+    dt = torch.float16 if in_dtype == "fp16" else torch.bfloat16
+    x = torch.from_numpy(w.x.reshape(w.M, w.K).view(np.int16)).view(dt).float()
+    xg = x.view(w.M, -1, group)
+    amax = xg.abs().amax(-1, keepdim=True).clamp_min(1e-10)
+    sc = amax / 448.0
+    ref = (xg / sc).clamp(-448.0, 448.0).to(torch.float8_e4m3fn).view(torch.uint8)
+    assert np.array_equal(s.reshape(w.M, -1), sc.squeeze(-1).numpy())
+    assert np.array_equal(q.reshape(w.M, -1, group), ref.numpy())
+
+
+# --------------------------------------------------------------------------
+# Fused SiLU-and-mul (P-9)
+# --------------------------------------------------------------------------
+
+def test_silu_mul_matches_torch_float64():
+    rng = np.random.default_rng(16)
+    g = np.concatenate([rng.standard_normal(400_000).astype(np.float32) * 3,
+                        np.float32([0.0, -0.0, 30.0, -30.0, 88.0, -88.0, 100.0, -100.0,
+                                    1e-30, -1e-30])])
+    u = rng.standard_normal(g.size).astype(np.float32)
+    ref = (torch.nn.functional.silu(torch.from_numpy(g).double())
+           * torch.from_numpy(u).double()).float().numpy()
+    got = oracle.silu_mul(g, u)
+    ulp = np.abs(got.view(np.int32).astype(np.int64) - ref.view(np.int32).astype(np.int64))
+    assert ulp.max() <= 1
+    assert (ulp == 0).mean() > 0.99999
+
+
+def test_fused_gate_is_first_half():
+    """silu(gate) * up with gate = columns [0, K), up = columns [K, 2K)."""
+    K = 128
+    x = np.zeros((1, 2 * K), np.float32)
+    x[0, :K] = 2.0           # gate
+    x[0, K:] = 1.0           # up
+    x[0, 3] = -1.0           # a negative gate entry
+    q, s = oracle.quant(inputs.bf16_bits(x), M=1, K=K, group=128, fused=True,
+                        scale_fmt="fp32")
+    silu2 = 2.0 / (1.0 + np.exp(-2.0))
+    silu_m1 = -1.0 / (1.0 + np.exp(1.0))
+    assert np.isclose(float(s.reshape(-1)[0]), silu2 / 448.0, rtol=1e-6)
+    assert int(q.reshape(-1)[0]) == 0x7E
+    assert int(q.reshape(-1)[3]) == int(brute_e4m3([silu_m1 / (silu2 / 448.0)])[0])
+    # swapping the halves changes the result, so the order is observable
+    xs = np.concatenate([x[:, K:], x[:, :K]], axis=1)
+    q2, s2 = oracle.quant(inputs.bf16_bits(xs), M=1, K=K, group=128, fused=True,
+                          scale_fmt="fp32")
+    assert not np.array_equal(s, s2)
+
+
+# --------------------------------------------------------------------------
+# Layouts and masked dispatch (P-10)
+# --------------------------------------------------------------------------
+
+def test_scale_layouts_are_one_table():
+    """row, col and packed hold the same exponents at their stated positions."""
+    M, K, G = 6, 5 * 128, 128            # ng = 5: a partial packed word; M_pad = 8
+    x = inputs.bf16_bits(inputs.normal((1, M, K), 21) * 10)
+    q_r, s_r = oracle.quant(x, M=M, K=K, group=G, scale_fmt="ue8m0", layout="row")
+    q_c, s_c = oracle.quant(x, M=M, K=K, group=G, scale_fmt="ue8m0", layout="col")
+    q_p, s_p = oracle.quant(x, M=M, K=K, group=G, scale_fmt="ue8m0", layout="packed")
+    assert np.array_equal(q_r, q_c) and np.array_equal(q_r, q_p)
+    row = s_r.reshape(M, 5)
+    col = s_c.reshape(5, 8)
+    assert np.array_equal(col[:, :M], row.T)
+    assert (col[:, M:] == 0xA5).all()                     # padding rows untouched
+    byts = s_p.reshape(2, 8).astype(np.int64)
+    for j in range(2):
+        for m in range(M):
+            w = int(byts[j, m]) & 0xFFFFFFFF
+            for b in range(4):
+                g = 4 * j + b
+                want = int(row[m, g]) if g < 5 else 0
+                assert (w >> (8 * b)) & 0xFF == want
+    assert (s_p.reshape(2, 8)[:, M:].view(np.uint32) == 0xA5A5A5A5).all()
+    # direct check of the row-major table against the exact ceiling
+    amax = np.maximum(np.abs(oracle.decode(x).reshape(M, 5, G)).max(-1), np.float32(1e-10))
+    assert np.array_equal(row.astype(np.int64), exact_ue8m0(amax).reshape(M, 5))
+    q_f, s_f = oracle.quant(x, M=M, K=K, group=G, scale_fmt="fp32", layout="col")
+    q_g, s_g = oracle.quant(x, M=M, K=K, group=G, scale_fmt="fp32", layout="row")
+    assert np.array_equal(s_f.reshape(5, 8)[:, :M], s_g.reshape(M, 5).T)
+
+
+def test_masked_rows_untouched_and_full_mask_equals_flat():
+    E, M, K = 3, 8, 256
+    x = inputs.bf16_bits(inputs.normal((E, M, 2 * K), 22))
+    mm = np.array([0, 5, 8], np.int32)
+    q, s = oracle.quant(x, E=E, M=M, K=K, group=128, fused=True, scale_fmt="ue8m0",
+                        layout="col", masked_m=mm)
+    q = q.reshape(E, M, K)
+    s = s.reshape(E, 2, M)
+    for e in range(E):
+        assert (q[e, mm[e]:] == 0xA5).all()
+        assert (s[e, :, mm[e]:] == 0xA5).all()
+        qf, sf = oracle.quant(x[e], M=M, K=K, group=128, fused=True, scale_fmt="ue8m0",
+                              layout="col")
+        assert np.array_equal(q[e, :mm[e]], qf.reshape(M, K)[:mm[e]])
+        assert np.array_equal(s[e, :, :mm[e]], sf.reshape(2, M)[:, :mm[e]])
+    # out-of-range counts are clamped to [0, M]
+    q2, _ = oracle.quant(x, E=E, M=M, K=K, group=128, fused=True, scale_fmt="ue8m0",
+                         layout="col", masked_m=np.array([-4, 5, 99], np.int32))
+    assert np.array_equal(q2, q.reshape(q2.shape))
+
+
+def test_oracle_rejects_unsupported_combinations():
+    x = np.zeros((1, 4, 256), np.uint16)
+    with pytest.raises(ValueError):
+        oracle.quant(x, M=4, K=256, group=128, out_dtype="int8", scale_fmt="ue8m0")
+    with pytest.raises(ValueError):
+        oracle.quant(x, M=4, K=256, group=128, scale_fmt="fp32", layout="packed")
+    nan = np.full((1, 4, 256), 0x7FC0, np.uint16)
+    with pytest.raises(ValueError):
+        oracle.quant(nan, M=4, K=256, group=128)
+
+
+# --------------------------------------------------------------------------
+# The seeded inputs are what their recipes say
+# --------------------------------------------------------------------------
+
+def test_inputs_are_deterministic_and_shaped():
+    a, b = inputs.tiny(), inputs.tiny()
+    assert np.array_equal(a.x, b.x) and a.x.shape == (1, 4, 256)
+    w = inputs.flat_hidden(M=256, K=7168)
+    x = oracle.decode(w.x).reshape(256, 7168)
+    for blk in range(2):
+        row, g = 128 * blk + (37 * blk) % 128, blk % 56
+        assert (x[row, g * 128:(g + 1) * 128] == 0).all()
+    assert (np.abs(x) > 20).mean() > 0.0005           # the x200 outliers exist
+    m = inputs.masked(E=4, M_max=64, K=128)
+    assert m.x.shape == (4, 64, 256) and m.masked_m.min() >= 0 and m.masked_m.max() <= 64
+    d = inputs.masked(E=8, M_max=16, K=128, decode=True)
+    assert set(np.unique(d.masked_m)) <= {0, 1} and d.expected_m == 1

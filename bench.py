@@ -1,0 +1,463 @@
+#!/usr/bin/env python
+"""Throughput of per-token-group activation quantization on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one pqg_quant call over the workload: load, optional SiLU-and-mul,
+group absmax, scale, quantize and scale store, all in one kernel.  The default
+workload is the flat quantization of a DeepSeek-V3 hidden state: bf16
+[8192, 7168] with outliers and all-zero groups, G = 128, E4M3 codes and UE8M0
+scales in the packed column-major layout.  Inputs are synthetic and seeded.
+They are resident in HBM before timing starts, and several buffer sets rotate so
+that each step's buffers have left the 126 MB L2 before they are reused.
+
+Rank 0 prints one JSON line.  ``value`` is effective HBM GB/s: the algorithmic
+bytes (input read, codes and scales written) of all ranks' steps divided by the
+slowest rank's device time.  Under torchrun each rank runs an independent
+replica on its own GPU (weak scaling, no data-path collective).  NCCL is only
+used for the barrier and the max over ranks of the timed interval.
+
+``--impl reference`` times the CPU oracle on bounded samples of the same
+workload instead, on rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "per-token-group quant effective HBM GB/s (% of 8 TB/s) and µs/call at M=1"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+L2_BYTES = 126 * 1024 * 1024
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic.json")
+
+
+def workloads():
+    from precision_activation_quantization_b200 import inputs
+    return {
+        "flat_hidden": lambda: inputs.flat_hidden(),
+        "flat_hidden_fp32": lambda: inputs.flat_hidden(layout="row", scale_fmt="fp32"),
+        "fused": lambda: inputs.fused(),
+        "masked": lambda: inputs.masked(),
+        "masked_decode": lambda: inputs.masked(decode=True),
+        "sweep_65536_bf16_e4m3_g128": lambda: inputs.sweep(65536),
+        "sweep_65536_fp16_int8_g32": lambda: inputs.sweep(65536, in_dtype="fp16",
+                                                          out_dtype="int8", group=32),
+    }
+
+
+def describe(w) -> dict:
+    shape = [w.E, w.M, 2 * w.K if w.fused else w.K] if w.E > 1 else \
+        [w.M, 2 * w.K if w.fused else w.K]
+    d = {"workload": w.name, "input_shape": shape, "in_dtype": w.in_dtype,
+         "out_dtype": w.out_dtype, "group": w.group,
+         "scales": f"{w.scale_fmt} {dict(row='row-major', col='column-major TMA-aligned', packed='UE8M0-packed column-major')[w.layout]}",
+         "fused_silu_mul": w.fused, "rows_quantized": w.rows,
+         "algorithmic_bytes_per_step": w.algorithmic_bytes()}
+    if w.masked_m is not None:
+        d["masked"] = {"experts": w.E, "M_max": w.M, "sum_masked_m": w.rows,
+                       "expected_m": w.expected_m}
+    return d
+
+
+def source_digest() -> str:
+    """sha256 over the CUDA sources, to tell whether stored ncu counters still apply."""
+    csrc = os.path.join(ROOT, "precision_activation_quantization_b200", "csrc")
+    h = hashlib.sha256()
+    for f in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
+    return h.hexdigest()
+
+
+def hbm_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def stored_traffic(name: str):
+    try:
+        with open(TRAFFIC_FILE) as f:
+            rec = json.load(f).get(name)
+        if rec and rec.get("source_sha256") == source_digest():
+            return rec["dram_bytes_per_launch"]
+    except Exception:
+        pass
+    return None
+
+
+# --------------------------------------------------------------------------
+# Clock sampling (NVML, polled during the timed region)
+# --------------------------------------------------------------------------
+
+class ClockSampler:
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x2: "applications_clocks_setting", 0x10: "sync_boost"}
+
+    def __init__(self, device_index: int):
+        self.samples, self.reasons = [], set()
+        self._stop = threading.Event()
+        self._thread = None
+        self.max_mhz = None
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            self._nvml = pynvml
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            try:
+                self._h = pynvml.nvmlDeviceGetHandleByUUID(
+                    uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+            except Exception:
+                self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._nvml = None
+
+    def _run(self):
+        n = self._nvml
+        get_reasons = getattr(n, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            n.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self._stop.is_set():
+            try:
+                self.samples.append(n.nvmlDeviceGetClockInfo(self._h, n.NVML_CLOCK_SM))
+                r = get_reasons(self._h)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self._nvml is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thread is not None:
+            self._thread.join()
+
+    def summary(self) -> dict:
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                    "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples),
+                "source": "NVML polled every ~2 ms during the timed region"}
+
+
+# --------------------------------------------------------------------------
+# The reference arm: the CPU oracle
+# --------------------------------------------------------------------------
+
+def run_reference(args, w) -> dict:
+    import oracle
+    rows = min(64, w.M)
+    live = [w.M if w.masked_m is None else int(np.clip(w.masked_m[e], 0, w.M))
+            for e in range(w.E)]
+    blocks = [(e, m0, min(rows, live[e] - m0)) for e in range(w.E)
+              for m0 in range(0, live[e], rows)]
+
+    def step(i):
+        e, m0, n = blocks[i % len(blocks)]
+        sub = w.with_(x=w.x[e:e + 1, m0:m0 + n], M=n, E=1, masked_m=None)
+        oracle.quant(sub.x, M=n, K=w.K, group=w.group, in_dtype=w.in_dtype,
+                     out_dtype=w.out_dtype, scale_fmt=w.scale_fmt, layout=w.layout,
+                     fused=w.fused)
+        return sub.algorithmic_bytes(), n
+
+    for i in range(args.warmup):
+        step(i)
+    total_bytes = total_rows = 0
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        b, n = step(args.warmup + i)
+        total_bytes += b
+        total_rows += n
+    dt = time.perf_counter() - t0
+    gbs = total_bytes / dt / 1e9
+    sample = (f"{rows}-row blocks of {w.name} (cycled), one per step, oracle single-threaded "
+              f"C at -O2")
+    return {"impl": "reference", "metric": METRIC, "value": gbs, "unit": "GB/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": dt * 1e3 / max(args.steps, 1), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": describe(w), "tokens_per_s": total_rows / dt,
+            "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def cpu_baseline(w, budget_s: float = 10.0) -> dict:
+    """The oracle as it stands, single-threaded, on whole copies of the workload
+    (masked: the live rows only) until about ``budget_s`` seconds have passed."""
+    import oracle
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        oracle.quant(w.x, E=w.E, M=w.M, K=w.K, group=w.group, in_dtype=w.in_dtype,
+                     out_dtype=w.out_dtype, scale_fmt=w.scale_fmt, layout=w.layout,
+                     fused=w.fused, masked_m=w.masked_m)
+        reps += 1
+        dt = time.perf_counter() - t0
+        if dt >= budget_s or reps >= 50:
+            break
+    return {"value": reps * w.algorithmic_bytes() / dt / 1e9, "unit": "GB/s", "cores": 1,
+            "kind": "oracle",
+            "sample": f"the whole {w.name} workload, {reps} time(s), {dt:.1f} s, one thread"}
+
+
+# --------------------------------------------------------------------------
+# Our arm
+# --------------------------------------------------------------------------
+
+def run_ours(args, w, rank: int, world: int, local_rank: int) -> dict | None:
+    import torch
+    import torch.distributed as dist
+    from precision_activation_quantization_b200 import pqg
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    sh = stream.cuda_stream
+
+    dt = torch.float16 if w.in_dtype == "fp16" else torch.bfloat16
+    x0 = torch.from_numpy(np.ascontiguousarray(w.x).view(np.int16)).view(dt).to(dev)
+    nbytes = pqg.pqg_scales_bytes(w.E, w.M, w.K, w.group, pqg.SCALE_FMTS[w.scale_fmt],
+                                  pqg.LAYOUTS[w.layout])
+    n_out = w.E * w.M * w.K
+    footprint = x0.numel() * 2 + n_out + nbytes
+    sets = max(1, min(8, -(-4 * L2_BYTES // footprint)))
+    xs = [x0] + [x0.clone() for _ in range(sets - 1)]
+    outs = [torch.empty(n_out, dtype=torch.uint8, device=dev) for _ in range(sets)]
+    scs = [torch.empty(max(nbytes, 1), dtype=torch.uint8, device=dev) for _ in range(sets)]
+    mm = None if w.masked_m is None else torch.from_numpy(w.masked_m).to(dev)
+    mm_ptr = None if mm is None else mm.data_ptr()
+    args_c = (w.M, w.E, w.K, w.group, pqg.IN_DTYPES[w.in_dtype], pqg.OUT_DTYPES[w.out_dtype],
+              pqg.SCALE_FMTS[w.scale_fmt], pqg.LAYOUTS[w.layout], int(w.fused))
+    ptrs = [(xs[i].data_ptr(), outs[i].data_ptr(), scs[i].data_ptr()) for i in range(sets)]
+
+    def launch(i):
+        a, b, c = ptrs[i % sets]
+        st = pqg.pqg_quant(a, b, c, *args_c, mm_ptr, w.expected_m, sh)
+        if st != pqg.PQG_OK:
+            raise pqg.PqgError(st)
+
+    def barrier():
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    for i in range(args.warmup):
+        launch(i)
+    barrier()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    launches0 = pqg.pqg_launch_count()
+    with ClockSampler(dev.index) as clocks:
+        start.record(stream)
+        for i in range(args.steps):
+            launch(args.warmup + i)
+        end.record(stream)
+        end.synchronize()
+    barrier()
+    launches = pqg.pqg_launch_count() - launches0
+    ms = start.elapsed_time(end)
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_step = ms / args.steps
+    bytes_step = w.algorithmic_bytes()
+    value = world * bytes_step * args.steps / (ms * 1e-3) / 1e9
+
+    # latency at M = 1 (same configuration, one row)
+    lat = latency_m1(w, dev, stream) if rank == 0 else None
+
+    # end to end: pinned host input -> device -> quantize -> codes/scales back
+    e2e = end_to_end(args, w, dev, stream, x0, outs[0], scs[0], mm_ptr, args_c, world)
+
+    del xs, outs, scs
+    torch.cuda.empty_cache()
+    if rank != 0:
+        return None
+
+    peak, peak_src = hbm_peak()
+    achieved = bytes_step / (ms_step * 1e-3) / 1e9
+    traffic = stored_traffic(w.name)
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic",
+        "config": dict(describe(w), l2=f"{sets} rotating buffer sets ({sets * footprint / 1e6:.0f} MB "
+                                       f"> 4 x 126 MB L2); each step reads a set last used "
+                                       f"{sets - 1} steps earlier",
+                       parallelism=f"{world} independent replica(s), no data-path collective"),
+        "pct_of_8tbs": 100.0 * value / world / NOMINAL_HBM_GBS,
+        "tokens_per_s": world * w.rows * args.steps / (ms * 1e-3),
+        "us_per_call_m1": lat,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "peak_source": peak_src,
+                     "traffic": traffic,
+                     "algorithmic_bytes_per_launch": bytes_step,
+                     "kernel": "pqg::quant_kernel (one launch per step)"},
+        "e2e": e2e,
+        "gpu_launches": launches,
+        "clocks": clocks.summary(),
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w)
+    return line
+
+
+def latency_m1(w, dev, stream) -> dict:
+    """µs per call at M = 1 (one row of the workload's shape and variant)."""
+    import torch
+    from precision_activation_quantization_b200 import pqg
+    width = 2 * w.K if w.fused else w.K
+    x = torch.zeros((1, width), dtype=torch.bfloat16 if w.in_dtype == "bf16" else torch.float16,
+                    device=dev)
+    x.normal_()
+    out = torch.empty(w.K, dtype=torch.uint8, device=dev)
+    nb = pqg.pqg_scales_bytes(1, 1, w.K, w.group, pqg.SCALE_FMTS[w.scale_fmt],
+                              pqg.LAYOUTS[w.layout])
+    sc = torch.empty(nb, dtype=torch.uint8, device=dev)
+    a = (x.data_ptr(), out.data_ptr(), sc.data_ptr(), 1, 1, w.K, w.group,
+         pqg.IN_DTYPES[w.in_dtype], pqg.OUT_DTYPES[w.out_dtype], pqg.SCALE_FMTS[w.scale_fmt],
+         pqg.LAYOUTS[w.layout], int(w.fused), None, 0)
+    s = torch.cuda.Stream(dev)
+    with torch.cuda.stream(s):
+        for _ in range(10):
+            pqg.pqg_quant(*a, s.cuda_stream)
+        n = 200
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            for _ in range(n):
+                pqg.pqg_quant(*a, s.cuda_stream)
+        g.replay()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = 10
+        e0.record(s)
+        for _ in range(reps):
+            g.replay()
+        e1.record(s)
+        e1.synchronize()
+        graph_us = e0.elapsed_time(e1) * 1e3 / (reps * n)
+        e0.record(s)
+        for _ in range(n):
+            pqg.pqg_quant(*a, s.cuda_stream)
+        e1.record(s)
+        e1.synchronize()
+        stream_us = e0.elapsed_time(e1) * 1e3 / n
+    del g
+    return {"graph": graph_us, "stream": stream_us,
+            "note": "1 x K row, same variant; graph = 200 launches captured in a CUDA graph "
+                    "(device time per call); stream = 200 back-to-back launches from Python"}
+
+
+def end_to_end(args, w, dev, stream, x_dev, out_dev, sc_dev, mm_ptr, args_c, world) -> dict:
+    """Same metric through the public API with host buffers: every step copies its
+    input from pinned host memory, quantizes, and reads codes and scales back."""
+    import torch
+    import torch.distributed as dist
+    from precision_activation_quantization_b200 import pqg
+    x_host = torch.from_numpy(np.ascontiguousarray(w.x).view(np.int16)).view(x_dev.dtype)
+    x_host = x_host.reshape(x_dev.shape).pin_memory()
+    out_host = torch.empty(out_dev.shape, dtype=torch.uint8).pin_memory()
+    sc_host = torch.empty(sc_dev.shape, dtype=torch.uint8).pin_memory()
+    steps = max(1, min(args.steps, 50))
+    sh = stream.cuda_stream
+
+    def step():
+        x_dev.copy_(x_host, non_blocking=True)
+        st = pqg.pqg_quant(x_dev.data_ptr(), out_dev.data_ptr(), sc_dev.data_ptr(), *args_c,
+                           mm_ptr, w.expected_m, sh)
+        if st != pqg.PQG_OK:
+            raise pqg.PqgError(st)
+        out_host.copy_(out_dev, non_blocking=True)
+        sc_host.copy_(sc_dev, non_blocking=True)
+
+    for _ in range(2):
+        step()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    e1.synchronize()
+    ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    return {"value": world * w.algorithmic_bytes() * steps / (ms * 1e-3) / 1e9, "unit": "GB/s",
+            "h2d_bytes_per_step": x_host.numel() * x_host.element_size(),
+            "d2h_bytes_per_step": out_host.numel() + sc_host.numel(),
+            "steps": steps, "ms_per_step": ms / steps}
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default="flat_hidden", choices=sorted(workloads()))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        w = workloads()[args.workload]()
+        print(json.dumps(run_reference(args, w)), flush=True)
+        return
+
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        w = workloads()[args.workload]()
+        line = run_ours(args, w, rank, world, local_rank)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

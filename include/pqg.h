@@ -1,0 +1,182 @@
+/*
+ * pqg — per-token-group activation quantization for NVIDIA B200 (sm_100a).
+ *
+ * C ABI of libpqg.so.  Plain pointers and sizes only; every buffer is owned by
+ * the caller, the library allocates no device or host memory, never
+ * synchronizes, and runs asynchronously on the stream it is given.
+ *
+ * The operation (sglang PR #30924 report, "[JIT] Trait-driven
+ * per_token_group_quant: unify the quant kernel family (flat + masked)"):
+ *   - 实现拆解 item 1 names the variant axes: input dtype (bf16/fp16), output
+ *     dtype (FP8-E4M3/INT8), group size, fp32 or UE8M0 scales, row- or
+ *     column-major scale layout, an optional fused silu_and_mul, and flat or
+ *     masked dispatch;
+ *   - 实现拆解 item 2 gives the masked dispatch its inputs masked_m and
+ *     expected_m;
+ *   - 关键源码片段, ref_fp8_ue8m0, gives the arithmetic: the absmax of each
+ *     1 x G group is floored at EPS; scale = amax / 448, or for UE8M0 the
+ *     power of two 2^e with e = biased exponent of fp32(amax / 448), plus one
+ *     when that quotient's mantissa is nonzero; codes = saturating cast of
+ *     x / scale clamped to [-448, 448];
+ *   - 风险与影响 (int8 码位差异) gives the INT8 variant with scale = amax / 127;
+ *     the same passage notes that callers no longer pass eps / min / max.
+ * The "FlashInfer GEMM 学习笔记" page (§6-7) states what the consumers of
+ * these codes want: block-scaled GEMMs read TMA-aligned packed scales, and
+ * grouped-masked GEMMs take a fixed expected_m plus a per-expert masked_m.
+ * "tf-kernel 安装与使用" (TeleFuser, 使用示例) splits a silu_and_mul input
+ * row into two halves of equal width.
+ *
+ * Numerics (every rounding to nearest, ties to even; no fast-math):
+ *   amax = max(max_i |x_i|, 1e-10f)                     (fp32)
+ *   FP32 scales : s = amax / 448 (E4M3) or amax / 127 (INT8), one IEEE division
+ *   UE8M0 scales: r = amax / 448; e = ((bits(r) >> 23) & 0xFF)
+ *                                     + ((bits(r) & 0x7FFFFF) != 0);
+ *                 s = 2^(e - 127); the stored byte is e
+ *   codes       : t = fp32(x / s) rounded once; E4M3 = nearest OCP E4M3 ("fn")
+ *                 value of t clamped to +-448 (zero keeps t's sign);
+ *                 INT8 = nearest integer of t clamped to [-128, 127]
+ *   fused       : x = silu(gate) * up computed in fp32 registers, gate being
+ *                 the first K columns of a 2K-wide input row, up the second;
+ *                 the product is never written to memory
+ * Codes and scales are bit-identical to that definition for every non-fused
+ * call.  The fused prologue uses the GPU's fast exponential, so its codes may
+ * move by one step where silu(gate)*up lies within a few fp32 ulps of a
+ * rounding midpoint.
+ */
+#ifndef PQG_H
+#define PQG_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Every entry point below is exported from libpqg.so; nothing else is. */
+#if defined(__GNUC__)
+#define PQG_API __attribute__((visibility("default")))
+#else
+#define PQG_API
+#endif
+
+/* Same type as cudaStream_t / CUstream.  NULL means the legacy default stream. */
+struct CUstream_st;
+typedef struct CUstream_st *pqg_stream_t;
+
+/* Status codes.  Every error is detected on the host before anything is
+ * launched, except PQG_ERR_CUDA, which reports a failed launch. */
+enum pqg_status {
+    PQG_OK = 0,
+    PQG_ERR_INVALID_ARG = -1, /* null pointer, bad size, unknown enum value     */
+    PQG_ERR_UNSUPPORTED = -2, /* valid values that do not combine (see below)  */
+    PQG_ERR_ALIGNMENT = -3,   /* a pointer misses its required alignment       */
+    PQG_ERR_CUDA = -4         /* the CUDA runtime reported an error; see
+                                 pqg_last_cuda_error()                          */
+};
+
+/* Element types. */
+enum pqg_dtype {
+    PQG_BF16 = 0, /* input: bfloat16                                  */
+    PQG_FP16 = 1, /* input: IEEE binary16                             */
+    PQG_E4M3 = 2, /* output: OCP FP8 E4M3 "fn" (max 448, no inf)       */
+    PQG_INT8 = 3  /* output: two's-complement int8                    */
+};
+
+/* Scale formats. */
+enum pqg_scale_fmt {
+    PQG_SCALE_FP32 = 0,  /* one float per group                        */
+    PQG_SCALE_UE8M0 = 1  /* one biased exponent byte e, scale 2^(e-127) */
+};
+
+/* Scale layouts, per expert.  ng = K / group; M_pad = M rounded up to a
+ * multiple of 4 (so that every column of the plane starts on a 16-byte
+ * boundary for fp32 scales and packed words).
+ *   PQG_ROW_MAJOR     : S[m][g]           element (m * ng + g)
+ *   PQG_COL_MAJOR_TMA : S[g][m]           element (g * M_pad + m); rows
+ *                       M..M_pad-1 are padding and are never written
+ *   PQG_UE8M0_PACKED  : W[j][m], int32    word (j * M_pad + m), j < ceil(ng/4);
+ *                       byte b (little-endian) of W[j][m] holds the exponent of
+ *                       group 4j + b; bytes for groups >= ng are written 0.
+ *                       UE8M0 only ("aligned" in the pages' trait list means
+ *                       ng % 4 == 0, i.e. no partial last word).
+ * Expert e's plane starts pqg_scales_bytes(1, M, K, ...) * e bytes into the
+ * buffer. */
+enum pqg_scale_layout {
+    PQG_ROW_MAJOR = 0,
+    PQG_COL_MAJOR_TMA = 1,
+    PQG_UE8M0_PACKED = 2
+};
+
+/*
+ * pqg_quant — quantize num_experts x M rows of K outputs each.
+ *
+ * in       device, read-only.  [num_experts][M][K] elements of in_dtype, or
+ *          [num_experts][M][2K] when fuse_silu_mul (row = gate | up).  Rows are
+ *          dense (row stride = K or 2K elements).  32-byte aligned.
+ * out      device.  [num_experts][M][K] one-byte codes (E4M3 or INT8).
+ *          16-byte aligned.
+ * scales   device.  pqg_scales_bytes(num_experts, M, K, group, scale_fmt,
+ *          scale_layout) bytes in the chosen layout.  4-byte aligned for fp32
+ *          scales and packed words, any alignment for UE8M0 bytes.
+ * M        rows per expert (with masked_m: the capacity M_max of each expert).
+ *          M >= 0; M == 0 launches nothing.
+ * num_experts  >= 1 (<= 65535).  With masked_m == NULL every expert's M rows
+ *          are quantized (num_experts == 1 is the flat dispatch).
+ * K        output elements per row, a positive multiple of group.
+ * group    G in {32, 64, 128}.
+ * in_dtype PQG_BF16 or PQG_FP16.   out_dtype PQG_E4M3 or PQG_INT8.
+ * scale_fmt, scale_layout   see above.  PQG_SCALE_UE8M0 requires PQG_E4M3, and
+ *          PQG_UE8M0_PACKED requires PQG_SCALE_UE8M0 (else PQG_ERR_UNSUPPORTED).
+ * fuse_silu_mul  nonzero: quantize silu(gate) * up (see the numerics above).
+ * masked_m device, int32[num_experts], or NULL.  Masked dispatch (grouped-masked
+ *          MoE): expert e quantizes only rows m < clamp(masked_m[e], 0, M); the
+ *          codes and scales of every other row are left untouched.  Read on the
+ *          device, so it may be produced by the preceding kernel on `stream`.
+ * expected_m  a hint for the masked grid: the typical masked_m value.  Results
+ *          never depend on it; <= 0 or > M means M.  Ignored when masked_m is
+ *          NULL.
+ * stream   CUDA stream the kernel is launched on.  The launch carries the
+ *          programmatic-dependent-launch attribute (see pqg_set_pdl); the kernel
+ *          waits for the preceding grid before its first global-memory access.
+ *
+ * Returns PQG_OK, or a negative pqg_status with nothing launched (except
+ * PQG_ERR_CUDA).  Limits: K <= 2^28, M * ceil(K / 512) < 2^31 and
+ * num_experts * M * K <= 2^40 (else PQG_ERR_INVALID_ARG).
+ * The output and scale buffers must not overlap the input.
+ */
+PQG_API int pqg_quant(const void *in, void *out, void *scales, int64_t M,
+              int64_t num_experts, int64_t K, int group, int in_dtype,
+              int out_dtype, int scale_fmt, int scale_layout, int fuse_silu_mul,
+              const int32_t *masked_m, int64_t expected_m, pqg_stream_t stream);
+
+/*
+ * pqg_scales_bytes — size in bytes of the scale buffer pqg_quant writes for
+ * these arguments (all experts, padding rows included).  Returns a negative
+ * pqg_status for arguments pqg_quant would reject.
+ */
+PQG_API int64_t pqg_scales_bytes(int64_t num_experts, int64_t M, int64_t K, int group,
+                         int scale_fmt, int scale_layout);
+
+/* Static, human-readable text for a status code. */
+PQG_API const char *pqg_status_string(int status);
+
+/* The cudaError_t of the last PQG_ERR_CUDA returned on the calling thread
+ * (0 if none). */
+PQG_API int pqg_last_cuda_error(void);
+
+/* Programmatic dependent launch (PDL) on (nonzero, the default) or off for
+ * later pqg_quant calls of this process.  Returns the previous setting. */
+PQG_API int pqg_set_pdl(int enable);
+
+/* Number of kernels this process has launched through pqg_quant so far. */
+PQG_API uint64_t pqg_launch_count(void);
+
+/* Library version string, e.g. "pqg 0.1.0 sm_100a". */
+PQG_API const char *pqg_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PQG_H */

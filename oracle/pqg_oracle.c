@@ -214,7 +214,6 @@ int pqgo_quant(const uint16_t *in, uint8_t *out, void *scales, int64_t E,
     if (layout < PQGO_ROW || layout > PQGO_PACKED) return -1;
     if (scale_ue8m0 && out_int8) return -1;       /* UE8M0 pairs with FMAX */
     if (layout == PQGO_PACKED && !scale_ue8m0) return -1;
-    if (masked_m && layout != PQGO_ROW && M % 4 != 0) return -1;
 
     const int64_t ng = K / G;
     const int64_t in_width = fused ? 2 * K : K;

@@ -1,0 +1,173 @@
+// C ABI of libpqg.so (declared in include/pqg.h): argument validation, scale
+// buffer geometry and dispatch into the kernel family.
+//
+// Every argument is checked on the host before anything is launched.  This
+// guards against the failure mode the sglang PR #30924 report (评论区精华 and
+// 风险与影响) records for its predecessor: negative dimension indices passed to
+// size_t accessors.  The library allocates nothing and never synchronizes.
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstdint>
+
+#include "pqg.h"
+#include "pqg_launch.cuh"
+
+namespace {
+
+thread_local int g_last_cuda_error = 0;
+std::atomic<int> g_pdl{1};
+std::atomic<uint64_t> g_launches{0};
+
+constexpr int64_t kMaxDevices = 64;
+std::atomic<int> g_sm_count[kMaxDevices];
+
+int64_t padded_rows(int64_t M) { return (M + 3) / 4 * 4; }
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Checks the enum values and sizes shared by pqg_quant and pqg_scales_bytes,
+// and returns the bytes of one expert's scale plane through *plane.
+int check_geometry(int64_t num_experts, int64_t M, int64_t K, int group, int scale_fmt,
+                   int scale_layout, int64_t *plane) {
+    if (scale_fmt != PQG_SCALE_FP32 && scale_fmt != PQG_SCALE_UE8M0) return PQG_ERR_INVALID_ARG;
+    if (scale_layout != PQG_ROW_MAJOR && scale_layout != PQG_COL_MAJOR_TMA &&
+        scale_layout != PQG_UE8M0_PACKED)
+        return PQG_ERR_INVALID_ARG;
+    if (group <= 0) return PQG_ERR_INVALID_ARG;
+    if (group != 32 && group != 64 && group != 128) return PQG_ERR_UNSUPPORTED;
+    if (scale_layout == PQG_UE8M0_PACKED && scale_fmt != PQG_SCALE_UE8M0)
+        return PQG_ERR_UNSUPPORTED;
+    if (num_experts < 1 || num_experts > 65535) return PQG_ERR_INVALID_ARG;
+    if (M < 0 || K <= 0 || K % group != 0) return PQG_ERR_INVALID_ARG;
+    // 2K-byte (4K fused) rows must fit the 32-bit row stride; strips per expert
+    // must fit a 32-bit index.
+    if (K > (int64_t{1} << 28)) return PQG_ERR_INVALID_ARG;
+    const int64_t segs = (K + pqg::kStripElems - 1) / pqg::kStripElems;
+    if (M > 0 && M >= (int64_t{1} << 31) / segs) return PQG_ERR_INVALID_ARG;
+    if (M * K > (int64_t{1} << 40) / num_experts) return PQG_ERR_INVALID_ARG;
+
+    const int64_t ng = K / group;
+    const int64_t elem = scale_fmt == PQG_SCALE_UE8M0 ? 1 : 4;
+    if (scale_layout == PQG_ROW_MAJOR)
+        *plane = M * ng * elem;
+    else if (scale_layout == PQG_COL_MAJOR_TMA)
+        *plane = ng * padded_rows(M) * elem;
+    else
+        *plane = (ng + 3) / 4 * padded_rows(M) * 4;
+    return PQG_OK;
+}
+
+bool overlaps(const void *a, int64_t na, const void *b, int64_t nb) {
+    const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+    return a0 < b0 + static_cast<uintptr_t>(nb) && b0 < a0 + static_cast<uintptr_t>(na);
+}
+
+}  // namespace
+
+namespace pqg {
+int sm_count(int device) {
+    if (device < 0 || device >= kMaxDevices) device = 0;
+    int n = g_sm_count[device].load(std::memory_order_relaxed);
+    if (n <= 0) {
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, device) != cudaSuccess ||
+            n <= 0)
+            n = 1;
+        g_sm_count[device].store(n, std::memory_order_relaxed);
+    }
+    return n;
+}
+}  // namespace pqg
+
+extern "C" {
+
+int64_t pqg_scales_bytes(int64_t num_experts, int64_t M, int64_t K, int group, int scale_fmt,
+                         int scale_layout) {
+    int64_t plane = 0;
+    const int st = check_geometry(num_experts, M, K, group, scale_fmt, scale_layout, &plane);
+    if (st != PQG_OK) return st;
+    return plane * num_experts;
+}
+
+int pqg_quant(const void *in, void *out, void *scales, int64_t M, int64_t num_experts, int64_t K,
+              int group, int in_dtype, int out_dtype, int scale_fmt, int scale_layout,
+              int fuse_silu_mul, const int32_t *masked_m, int64_t expected_m,
+              pqg_stream_t stream) {
+    if (in_dtype != PQG_BF16 && in_dtype != PQG_FP16) return PQG_ERR_INVALID_ARG;
+    if (out_dtype != PQG_E4M3 && out_dtype != PQG_INT8) return PQG_ERR_INVALID_ARG;
+    int64_t plane = 0;
+    const int st = check_geometry(num_experts, M, K, group, scale_fmt, scale_layout, &plane);
+    if (st != PQG_OK) return st;
+    if (scale_fmt == PQG_SCALE_UE8M0 && out_dtype != PQG_E4M3) return PQG_ERR_UNSUPPORTED;
+    if (M == 0) return PQG_OK;
+
+    if (in == nullptr || out == nullptr || scales == nullptr) return PQG_ERR_INVALID_ARG;
+    if (!aligned(in, 32) || !aligned(out, 16)) return PQG_ERR_ALIGNMENT;
+    if (scale_fmt == PQG_SCALE_FP32 || scale_layout == PQG_UE8M0_PACKED) {
+        if (!aligned(scales, 4)) return PQG_ERR_ALIGNMENT;
+    }
+    if (masked_m != nullptr && !aligned(masked_m, 4)) return PQG_ERR_ALIGNMENT;
+
+    const int64_t in_row_bytes = K * 2 * (fuse_silu_mul ? 2 : 1);
+    const int64_t in_bytes = num_experts * M * in_row_bytes;
+    const int64_t out_bytes = num_experts * M * K;
+    if (overlaps(in, in_bytes, out, out_bytes) || overlaps(in, in_bytes, scales, plane * num_experts) ||
+        overlaps(out, out_bytes, scales, plane * num_experts))
+        return PQG_ERR_INVALID_ARG;
+
+    pqg::LaunchArgs a;
+    a.p.in = static_cast<const uint8_t *>(in);
+    a.p.out = static_cast<uint8_t *>(out);
+    a.p.scales = static_cast<uint8_t *>(scales);
+    a.p.masked_m = masked_m;
+    a.p.in_expert_bytes = M * in_row_bytes;
+    a.p.out_expert_bytes = M * K;
+    a.p.scale_expert_bytes = plane;
+    a.p.M = static_cast<uint32_t>(M);
+    a.p.K = static_cast<uint32_t>(K);
+    a.p.in_row_bytes = static_cast<uint32_t>(in_row_bytes);
+    a.p.ng = static_cast<uint32_t>(K / group);
+    a.p.segs = static_cast<uint32_t>((K + pqg::kStripElems - 1) / pqg::kStripElems);
+    a.p.mpad = static_cast<uint32_t>(padded_rows(M));
+    a.p.layout = static_cast<uint32_t>(scale_layout);
+    a.experts = static_cast<uint32_t>(num_experts);
+    a.grid_rows = static_cast<uint32_t>(
+        (masked_m != nullptr && expected_m > 0 && expected_m < M) ? expected_m : M);
+    a.group = group;
+    a.kind = scale_fmt == PQG_SCALE_UE8M0 ? pqg::Kind::E4M3_UE8M0
+             : out_dtype == PQG_INT8      ? pqg::Kind::INT8_FP32
+                                          : pqg::Kind::E4M3_FP32;
+    a.fused = fuse_silu_mul != 0;
+    a.pdl = g_pdl.load(std::memory_order_relaxed) != 0;
+    a.stream = reinterpret_cast<cudaStream_t>(stream);
+
+    const cudaError_t err = in_dtype == PQG_BF16 ? pqg::launch_bf16(a) : pqg::launch_fp16(a);
+    if (err != cudaSuccess) {
+        g_last_cuda_error = static_cast<int>(err);
+        (void)cudaGetLastError();  // the error is reported here; do not leave it sticky
+        return PQG_ERR_CUDA;
+    }
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return PQG_OK;
+}
+
+const char *pqg_status_string(int status) {
+    switch (status) {
+        case PQG_OK: return "ok";
+        case PQG_ERR_INVALID_ARG: return "invalid argument";
+        case PQG_ERR_UNSUPPORTED: return "unsupported combination of arguments";
+        case PQG_ERR_ALIGNMENT: return "pointer misaligned";
+        case PQG_ERR_CUDA: return "CUDA runtime error";
+    }
+    return "unknown status";
+}
+
+int pqg_last_cuda_error(void) { return g_last_cuda_error; }
+
+int pqg_set_pdl(int enable) { return g_pdl.exchange(enable != 0 ? 1 : 0); }
+
+uint64_t pqg_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+const char *pqg_version(void) { return "pqg 0.1.0 sm_100a"; }
+
+}  // extern "C"

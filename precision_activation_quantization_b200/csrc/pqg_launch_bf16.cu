@@ -1,0 +1,6 @@
+// Instantiates the bf16-input half of the kernel family (18 variants).
+#include "pqg_launch.cuh"
+
+namespace pqg {
+cudaError_t launch_bf16(const LaunchArgs &a) { return launch_dtype<__nv_bfloat16>(a); }
+}  // namespace pqg

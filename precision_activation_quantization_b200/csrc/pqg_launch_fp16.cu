@@ -1,0 +1,6 @@
+// Instantiates the fp16-input half of the kernel family (18 variants).
+#include "pqg_launch.cuh"
+
+namespace pqg {
+cudaError_t launch_fp16(const LaunchArgs &a) { return launch_dtype<__half>(a); }
+}  // namespace pqg

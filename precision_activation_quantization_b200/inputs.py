@@ -16,10 +16,16 @@ items 1-2.
 """
 from __future__ import annotations
 
+import concurrent.futures as cf
 import dataclasses
+import os
 
 import numpy as np
 import torch
+
+# Draws are made in fixed chunks, each from its own generator seeded by
+# (seed, chunk index), so the values do not depend on how many threads run.
+_CHUNK = 1 << 22
 
 
 def bf16_bits(f32: np.ndarray) -> np.ndarray:
@@ -37,20 +43,37 @@ def to_bits(f32: np.ndarray, in_dtype: str) -> np.ndarray:
     return f16_bits(f32) if in_dtype == "fp16" else bf16_bits(f32)
 
 
+def _chunked(shape, seed: int, fill) -> np.ndarray:
+    out = np.empty(int(np.prod(shape)), np.float32)
+    n_chunks = (out.size + _CHUNK - 1) // _CHUNK
+
+    def work(i):
+        rng = np.random.default_rng([seed, i])
+        fill(rng, out[i * _CHUNK:(i + 1) * _CHUNK])
+
+    if n_chunks <= 1:
+        for i in range(n_chunks):
+            work(i)
+    else:
+        with cf.ThreadPoolExecutor(max_workers=min(16, os.cpu_count() or 1)) as ex:
+            list(ex.map(work, range(n_chunks)))
+    return out.reshape(shape)
+
+
 def normal(shape, seed: int, scale: float = 1.0) -> np.ndarray:
-    rng = np.random.default_rng(seed)
-    x = rng.standard_normal(size=shape, dtype=np.float32)
-    if scale != 1.0:
-        x *= np.float32(scale)
-    return x
+    def fill(rng, view):
+        rng.standard_normal(out=view, dtype=np.float32)
+        if scale != 1.0:
+            view *= np.float32(scale)
+    return _chunked(shape, seed, fill)
 
 
 def laplace(shape, seed: int) -> np.ndarray:
     """Laplace(0, 1) draws by the inverse CDF of seeded uniforms."""
-    rng = np.random.default_rng(seed)
-    u = rng.random(size=shape, dtype=np.float64) - 0.5
-    x = -np.sign(u) * np.log1p(-2.0 * np.abs(u))
-    return x.astype(np.float32)
+    def fill(rng, view):
+        u = rng.random(size=view.size, dtype=np.float64) - 0.5
+        view[:] = -np.sign(u) * np.log1p(-2.0 * np.abs(u))
+    return _chunked(shape, seed, fill)
 
 
 @dataclasses.dataclass

@@ -1,0 +1,193 @@
+"""Helpers shared by the GPU parity tests: run a workload through the C ABI and
+through the oracle, and compare the results.
+
+The kernel's output and scale buffers are filled with a sentinel byte first and
+carry a guard band past their end, so that writes to rows the call must not
+touch, or writes past the buffer, show up as changed sentinel bytes.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle
+from precision_activation_quantization_b200 import pqg
+
+SENTINEL = 0xA5
+GUARD = 4096
+
+
+def _torch_input(w):
+    dt = torch.float16 if w.in_dtype == "fp16" else torch.bfloat16
+    return torch.from_numpy(np.ascontiguousarray(w.x).view(np.int16)).view(dt).cuda()
+
+
+def run_gpu(w, *, expected_m=None, stream=None, x_dev=None):
+    """Run ``w`` through pqg_quant; returns (codes uint8 [E*M*K], scale bytes)."""
+    x = _torch_input(w) if x_dev is None else x_dev
+    n_out = w.E * w.M * w.K
+    nbytes = pqg.pqg_scales_bytes(w.E, w.M, w.K, w.group, pqg.SCALE_FMTS[w.scale_fmt],
+                                  pqg.LAYOUTS[w.layout])
+    assert nbytes >= 0
+    out = torch.full((n_out + GUARD,), SENTINEL, dtype=torch.uint8, device="cuda")
+    sc = torch.full((nbytes + GUARD,), SENTINEL, dtype=torch.uint8, device="cuda")
+    mm = None if w.masked_m is None else torch.from_numpy(np.asarray(w.masked_m, np.int32)).cuda()
+    s = stream if stream is not None else torch.cuda.current_stream()
+    st = pqg.pqg_quant(x.data_ptr(), out.data_ptr(), sc.data_ptr(), w.M, w.E, w.K, w.group,
+                       pqg.IN_DTYPES[w.in_dtype], pqg.OUT_DTYPES[w.out_dtype],
+                       pqg.SCALE_FMTS[w.scale_fmt], pqg.LAYOUTS[w.layout], int(w.fused),
+                       None if mm is None else mm.data_ptr(),
+                       w.expected_m if expected_m is None else expected_m, s.cuda_stream)
+    assert st == pqg.PQG_OK, pqg.pqg_status_string(st)
+    torch.cuda.synchronize()
+    out_h, sc_h = out.cpu().numpy(), sc.cpu().numpy()
+    assert (out_h[n_out:] == SENTINEL).all(), "codes written past the end of the buffer"
+    assert (sc_h[nbytes:] == SENTINEL).all(), "scales written past the end of the buffer"
+    return out_h[:n_out], sc_h[:nbytes]
+
+
+def run_oracle(w):
+    """The oracle's (codes uint8 [E*M*K], scale bytes), sentinel-filled like run_gpu."""
+    q, s = oracle.quant(w.x, E=w.E, M=w.M, K=w.K, group=w.group, in_dtype=w.in_dtype,
+                        out_dtype=w.out_dtype, scale_fmt=w.scale_fmt, layout=w.layout,
+                        fused=w.fused, masked_m=w.masked_m, fill=SENTINEL)
+    return q.reshape(-1), s.view(np.uint8).reshape(-1)
+
+
+def assert_same(gpu, ref, what):
+    if np.array_equal(gpu, ref):
+        return
+    bad = np.flatnonzero(gpu != ref)
+    raise AssertionError(f"{what}: {bad.size} of {ref.size} bytes differ; first at "
+                         f"{bad[:8].tolist()} gpu={gpu[bad[:8]].tolist()} "
+                         f"oracle={ref[bad[:8]].tolist()}")
+
+
+def check_exact(w, **kw):
+    """Non-fused contract: codes, scales and untouched bytes are bit-identical."""
+    gq, gs = run_gpu(w, **kw)
+    rq, rs = run_oracle(w)
+    assert_same(gq, rq, f"{w.name} codes")
+    assert_same(gs, rs, f"{w.name} scales")
+    return gq, gs
+
+
+# --------------------------------------------------------------------------
+# The fused tolerance contract
+# --------------------------------------------------------------------------
+
+def _e4m3_values() -> np.ndarray:
+    codes = torch.arange(256, dtype=torch.int32).to(torch.uint8)
+    return codes.view(torch.float8_e4m3fn).double().numpy()
+
+
+E4M3 = _e4m3_values()
+_FINITE = np.sort(np.unique(E4M3[~np.isnan(E4M3)]))     # -448 .. 448, one zero
+E4M3_RANK = np.searchsorted(_FINITE, np.nan_to_num(E4M3))  # code -> position
+
+
+def _scale_planes(w, sbytes):
+    """Per-group scales as float64 [E, M, ng] from the scale buffer, and the
+    matching UE8M0 byte table (or None)."""
+    ng, mpad = w.K // w.group, (w.M + 3) // 4 * 4
+    if w.scale_fmt == "ue8m0":
+        if w.layout == "packed":
+            words = sbytes.reshape(w.E, (ng + 3) // 4, mpad, 4)
+            e8 = words.transpose(0, 2, 1, 3).reshape(w.E, mpad, -1)[:, :w.M, :ng]
+        elif w.layout == "col":
+            e8 = sbytes.reshape(w.E, ng, mpad)[:, :, :w.M].transpose(0, 2, 1)
+        else:
+            e8 = sbytes.reshape(w.E, w.M, ng)
+        return np.exp2(e8.astype(np.float64) - 127.0), e8
+    f = sbytes.view(np.float32)
+    if w.layout == "col":
+        f = f.reshape(w.E, ng, mpad)[:, :, :w.M].transpose(0, 2, 1)
+    else:
+        f = f.reshape(w.E, w.M, ng)
+    return f.astype(np.float64), None
+
+
+def check_fused(w, *, max_flip_frac=1e-4, rel_tol=7e-2, **kw):
+    """Fused contract: scales equal (fp32 within 1 ulp; UE8M0 equal unless the
+    oracle's amax/448 is within 2^-20 of a power of two); codes equal except for
+    at most ``max_flip_frac`` of elements that move by one step; every element's
+    dequantized value within ``rel_tol`` of the oracle's silu(gate)*up."""
+    gq, gs = run_gpu(w, **kw)
+    rq, rs = run_oracle(w)
+    E, M, K, G = w.E, w.M, w.K, w.group
+    rows = np.full(E, M) if w.masked_m is None else np.clip(w.masked_m, 0, M)
+    live = np.arange(M)[None, :] < rows[:, None]                       # [E, M]
+
+    # untouched rows and padding must be byte-identical (sentinels)
+    gq3, rq3 = gq.reshape(E, M, K), rq.reshape(E, M, K)
+    assert_same(gq3[~live], rq3[~live], f"{w.name} masked-off codes")
+    g_sc, g_e8 = _scale_planes(w, gs)
+    r_sc, r_e8 = _scale_planes(w, rs)
+    # scale bytes outside live (row, group) cells must be untouched
+    ng, mpad = K // G, (M + 3) // 4 * 4
+    idx = np.arange(gs.size)
+    if w.layout == "packed":
+        word = idx // 4
+        m_of, e_of = word % mpad, word // (((ng + 3) // 4) * mpad)
+    else:
+        elem = idx // (1 if w.scale_fmt == "ue8m0" else 4)
+        if w.layout == "col":
+            m_of, e_of = elem % mpad, elem // (ng * mpad)
+        else:
+            m_of, e_of = (elem // ng) % M, elem // (M * ng)
+    inside = m_of < rows[e_of]
+    assert_same(gs[~inside], rs[~inside], f"{w.name} untouched scale bytes")
+    if w.layout == "packed":
+        j = (idx // 4 // mpad) % ((ng + 3) // 4)
+        pad = inside & (4 * j + idx % 4 >= ng)
+        assert (gs[pad] == 0).all(), "packed padding bytes must be 0"
+
+    # the oracle's fused values, for the dequant bound and the flip exemption
+    import oracle as _o
+    xf = _o.decode(w.x, w.in_dtype).reshape(E, M, 2 * K)
+    y = _o.silu_mul(xf[..., :K], xf[..., K:]).astype(np.float64)      # [E, M, K]
+    yg = y.reshape(E, M, K // G, G)
+    amax = np.maximum(np.abs(yg).max(-1), 1e-10)
+
+    g_sc, r_sc = g_sc[live], r_sc[live]                                # [n_live, ng]
+    if g_e8 is not None:
+        g_e8, r_e8 = g_e8[live].astype(np.int64), r_e8[live].astype(np.int64)
+        scale_diff = g_e8 != r_e8
+        r = (amax[live] / 448.0)
+        near_pow2 = np.abs(r / np.exp2(np.round(np.log2(r))) - 1.0) < 2.0 ** -20
+        assert (~scale_diff | near_pow2).all(), \
+            f"{w.name}: {int((scale_diff & ~near_pow2).sum())} UE8M0 bytes differ away from a power of two"
+    else:
+        ulps = np.abs(g_sc.astype(np.float32).view(np.int32).astype(np.int64)
+                      - r_sc.astype(np.float32).view(np.int32).astype(np.int64))
+        assert ulps.max(initial=0) <= 1, f"{w.name}: fp32 scale off by {ulps.max()} ulp"
+        scale_diff = ulps > 0
+
+    gcodes = gq3[live].reshape(-1, K // G, G)
+    rcodes = rq3[live].reshape(-1, K // G, G)
+    same_scale = ~scale_diff
+    diff = (gcodes != rcodes) & same_scale[..., None]
+    n_el = gcodes.size
+    if w.out_dtype == "int8":
+        step = np.abs(gcodes.view(np.int8).astype(np.int64) - rcodes.view(np.int8).astype(np.int64))
+    else:
+        step = np.abs(E4M3_RANK[gcodes].astype(np.int64) - E4M3_RANK[rcodes].astype(np.int64))
+    assert (step[diff] <= 1).all(), f"{w.name}: a code moved by more than one step"
+    frac = diff.sum() / max(n_el, 1)
+    assert frac <= max_flip_frac, f"{w.name}: {frac:.2e} of codes differ (> {max_flip_frac})"
+
+    # dequantized GPU value vs the oracle's y, per element
+    vals = (gcodes.view(np.int8).astype(np.float64) if w.out_dtype == "int8"
+            else E4M3[gcodes])
+    deq = vals * g_sc[..., None]
+    yl = y[live].reshape(-1, K // G, G)
+    t = np.abs(yl) / g_sc[..., None]
+    err = np.abs(deq - yl)
+    if w.out_dtype == "int8":
+        assert (err <= (0.5 + 1.0) * g_sc[..., None]).all()
+    else:
+        big = t >= 2.0 ** -6
+        assert (err[big] <= rel_tol * np.abs(yl[big])).all(), f"{w.name}: dequant error"
+        small_bound = np.broadcast_to(g_sc[..., None], t.shape)[~big] * 2.0 ** -9
+        assert (err[~big] <= small_bound).all(), f"{w.name}: dequant error near zero"
+    return dict(flip_frac=float(frac), scale_flips=int(scale_diff.sum()))

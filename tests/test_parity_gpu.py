@@ -1,0 +1,241 @@
+"""GPU parity: the CUDA path through the C ABI against the CPU oracle.
+
+Non-fused calls must match bit for bit: codes, fp32 scales, UE8M0 bytes, packed
+words, and every byte the call must not touch (sentinels).  Fused calls follow
+the tolerance contract in ``gpu_parity.check_fused``.  Sizes run from a single
+group to the full workloads, with ragged tails where K is not a multiple of
+512 and M is not a multiple of 4.
+"""
+import numpy as np
+import pytest
+import torch
+
+from precision_activation_quantization_b200 import inputs, pqg
+from gpu_parity import SENTINEL, assert_same, check_exact, check_fused, run_gpu, run_oracle
+
+pytestmark = pytest.mark.gpu
+
+KINDS = [  # (out_dtype, scale_fmt, layout)
+    ("e4m3", "fp32", "row"), ("e4m3", "fp32", "col"),
+    ("e4m3", "ue8m0", "row"), ("e4m3", "ue8m0", "col"), ("e4m3", "ue8m0", "packed"),
+    ("int8", "fp32", "row"), ("int8", "fp32", "col"),
+]
+
+
+def hard_input(shape, seed, in_dtype="bf16"):
+    """N(0,1) rows with per-row magnitudes over many binades, all-zero groups of
+    32, -0.0 entries, outliers and subnormal inputs."""
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal(shape).astype(np.float32)
+    lo, hi = (-20, 10) if in_dtype == "bf16" else (-12, 6)
+    x *= np.exp2(rng.uniform(lo, hi, shape[:-1] + (1,))).astype(np.float32)
+    flat = x.reshape(-1, 32)
+    flat[rng.random(flat.shape[0]) < 1 / 16] = 0.0
+    x[rng.random(shape) < 0.01] = -0.0
+    out = rng.random(shape) < 0.005
+    x[out] *= np.float32(300.0 if in_dtype == "bf16" else 30.0)
+    sub = rng.random(shape) < 0.005
+    x[sub] = (np.float32(3e-39) if in_dtype == "bf16" else np.float32(3e-6)) * np.sign(
+        rng.standard_normal(int(sub.sum()))).astype(np.float32)
+    if in_dtype == "fp16":
+        x = np.clip(x, -60000, 60000)
+    return inputs.to_bits(x, in_dtype)
+
+
+def make(M, K, G, kind, in_dtype="bf16", fused=False, E=1, seed=0, masked_m=None,
+         expected_m=0):
+    out_dtype, fmt, layout = kind
+    width = 2 * K if fused else K
+    x = hard_input((E, M, width), seed, in_dtype)
+    return inputs.Workload(f"M{M}_K{K}_G{G}_{in_dtype}_{'_'.join(kind)}{'_fused' if fused else ''}",
+                           x, M=M, K=K, group=G, E=E, in_dtype=in_dtype, out_dtype=out_dtype,
+                           scale_fmt=fmt, layout=layout, fused=fused, masked_m=masked_m,
+                           expected_m=expected_m)
+
+
+# --------------------------------------------------------------------------
+# every variant on ragged shapes
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("kind", KINDS, ids=lambda k: "_".join(k))
+@pytest.mark.parametrize("G", [32, 64, 128])
+@pytest.mark.parametrize("in_dtype", ["bf16", "fp16"])
+def test_flat_variants_bit_exact(kind, G, in_dtype):
+    for M, K in [(37, 640), (5, 128), (130, 2048), (1, 7168)]:
+        check_exact(make(M, K, G, kind, in_dtype, seed=M + K + G))
+
+
+@pytest.mark.parametrize("kind", KINDS, ids=lambda k: "_".join(k))
+@pytest.mark.parametrize("G", [32, 128])
+@pytest.mark.parametrize("in_dtype", ["bf16", "fp16"])
+def test_fused_variants_within_contract(kind, G, in_dtype):
+    for M, K in [(37, 640), (130, 2048)]:
+        check_fused(make(M, K, G, kind, in_dtype, fused=True, seed=M + K + G + 1),
+                    max_flip_frac=1e-3)   # small samples: a handful of flips
+
+
+@pytest.mark.parametrize("kind", KINDS, ids=lambda k: "_".join(k))
+def test_masked_variants(kind):
+    E, M, K = 5, 37, 640
+    mm = np.array([0, 37, 1, 99, -3], np.int32)          # empty, full, one, >M, <0
+    for fused in (False, True):
+        w = make(M, K, 128, kind, fused=fused, E=E, seed=3, masked_m=mm, expected_m=8)
+        if fused:
+            check_fused(w, max_flip_frac=1e-3)
+        else:
+            check_exact(w)
+
+
+# --------------------------------------------------------------------------
+# exhaustive input values
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("in_dtype", ["bf16", "fp16"])
+@pytest.mark.parametrize("kind", [("e4m3", "fp32", "row"), ("e4m3", "ue8m0", "row"),
+                                  ("int8", "fp32", "row")], ids=lambda k: "_".join(k))
+@pytest.mark.parametrize("carrier", [1.0, 448.0, 3.0e-3, 1000.0])
+def test_every_input_value_in_a_carrier_group(in_dtype, kind, carrier):
+    """Each finite bf16/fp16 value sits in its own 128-group next to a carrier."""
+    bits = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    import oracle
+    vals = oracle.decode(bits, in_dtype)
+    bits = bits[np.isfinite(vals)]
+    n = bits.size
+    cb = inputs.to_bits(np.float32([carrier]), in_dtype)[0]
+    x = np.full((1, n, 128), cb, np.uint16)
+    x[0, :, 0] = bits
+    x[0, :, 77] = bits ^ 0x8000                          # the negated value too
+    out_dtype, fmt, layout = kind
+    w = inputs.Workload("exhaustive", x, M=n, K=128, group=128, in_dtype=in_dtype,
+                        out_dtype=out_dtype, scale_fmt=fmt, layout=layout)
+    check_exact(w)
+
+
+# --------------------------------------------------------------------------
+# the full workloads
+# --------------------------------------------------------------------------
+
+def test_tiny_workload():
+    check_exact(inputs.tiny())
+
+
+@pytest.mark.parametrize("layout,fmt", [("packed", "ue8m0"), ("row", "fp32"), ("col", "ue8m0"),
+                                        ("col", "fp32")])
+def test_flat_hidden_full_size(layout, fmt):
+    check_exact(inputs.flat_hidden(layout=layout, scale_fmt=fmt))
+
+
+def test_fused_full_size():
+    stats = check_fused(inputs.fused())
+    print("fused flips", stats)
+
+
+def test_masked_full_size():
+    w = inputs.masked()
+    stats = check_fused(w)
+    print("masked flips", stats)
+
+
+def test_masked_decode():
+    check_fused(inputs.masked(decode=True))
+
+
+@pytest.mark.parametrize("M", [1, 16, 128, 1024, 16384])
+@pytest.mark.parametrize("in_dtype", ["bf16", "fp16"])
+@pytest.mark.parametrize("G", [32, 64, 128])
+@pytest.mark.parametrize("out_dtype", ["int8", "e4m3"])
+def test_sweep(M, in_dtype, G, out_dtype):
+    check_exact(inputs.sweep(M, in_dtype=in_dtype, group=G, out_dtype=out_dtype))
+
+
+@pytest.mark.parametrize("in_dtype,out_dtype,G", [("bf16", "e4m3", 128), ("fp16", "int8", 32)])
+def test_sweep_largest(in_dtype, out_dtype, G):
+    check_exact(inputs.sweep(65536, in_dtype=in_dtype, group=G, out_dtype=out_dtype))
+
+
+# --------------------------------------------------------------------------
+# dispatch properties
+# --------------------------------------------------------------------------
+
+def test_expected_m_does_not_change_results():
+    E, M, K = 6, 64, 1024
+    mm = np.array([64, 3, 0, 17, 64, 40], np.int32)
+    w = make(M, K, 128, ("e4m3", "ue8m0", "col"), fused=True, E=E, seed=9, masked_m=mm)
+    ref = run_gpu(w, expected_m=1)
+    for em in (0, 8, 30, 64, 1000):
+        got = run_gpu(w, expected_m=em)
+        assert_same(got[0], ref[0], f"codes, expected_m={em}")
+        assert_same(got[1], ref[1], f"scales, expected_m={em}")
+
+
+def test_full_mask_equals_batched_flat():
+    E, M, K = 3, 20, 512
+    w = make(M, K, 64, ("e4m3", "fp32", "col"), E=E, seed=11)
+    flat = run_gpu(w)
+    masked = run_gpu(w.with_(masked_m=np.full(E, M, np.int32), expected_m=5))
+    assert_same(masked[0], flat[0], "codes")
+    assert_same(masked[1], flat[1], "scales")
+
+
+def test_pdl_off_matches_on():
+    w = make(33, 1536, 128, ("e4m3", "ue8m0", "packed"), seed=12)
+    on = run_gpu(w)
+    prev = pqg.pqg_set_pdl(False)
+    try:
+        off = run_gpu(w)
+    finally:
+        pqg.pqg_set_pdl(prev)
+    assert_same(off[0], on[0], "codes")
+    assert_same(off[1], on[1], "scales")
+
+
+def test_side_stream_and_graph_replay():
+    w = make(64, 2048, 128, ("e4m3", "fp32", "row"), seed=13)
+    ref_q, ref_s = run_oracle(w)
+    x = torch.from_numpy(w.x.view(np.int16)).view(torch.bfloat16).cuda()
+    out = torch.empty(64 * 2048, dtype=torch.uint8, device="cuda")
+    sc = torch.empty(64 * 16 * 4, dtype=torch.uint8, device="cuda")
+    s = torch.cuda.Stream()
+
+    def launch():
+        st = pqg.pqg_quant(x.data_ptr(), out.data_ptr(), sc.data_ptr(), 64, 1, 2048, 128,
+                           pqg.PQG_BF16, pqg.PQG_E4M3, pqg.PQG_SCALE_FP32, pqg.PQG_ROW_MAJOR, 0,
+                           None, 0, s.cuda_stream)
+        assert st == pqg.PQG_OK
+
+    with torch.cuda.stream(s):
+        launch()
+    torch.cuda.synchronize()
+    assert_same(out.cpu().numpy(), ref_q, "side-stream codes")
+    out.fill_(0)
+    sc.fill_(0)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        launch()
+    g.replay()
+    torch.cuda.synchronize()
+    assert_same(out.cpu().numpy(), ref_q, "graph codes")
+    assert_same(sc.cpu().numpy(), ref_s, "graph scales")
+
+
+def test_repeatable_and_launch_counted():
+    w = inputs.sweep(128, group=64)
+    before = pqg.pqg_launch_count()
+    a = run_gpu(w)
+    b = run_gpu(w)
+    assert pqg.pqg_launch_count() == before + 2
+    assert_same(a[0], b[0], "codes")
+    assert_same(a[1], b[1], "scales")
+
+
+def test_torch_helper_matches_raw_call():
+    w = inputs.flat_hidden(M=256, K=7168)
+    x = torch.from_numpy(w.x.reshape(256, 7168).view(np.int16)).view(torch.bfloat16).cuda()
+    q, s = pqg.quant(x, group=128, scale_fmt="ue8m0", layout="packed")
+    torch.cuda.synchronize()
+    rq, rs = run_oracle(w)
+    assert_same(q.view(torch.uint8).cpu().numpy().reshape(-1), rq, "codes")
+    assert_same(s.view(torch.uint8).cpu().numpy().reshape(-1), rs, "scales")
+    with pytest.raises(pqg.PqgError):
+        pqg.quant(x, group=128, out_dtype="int8", scale_fmt="ue8m0")

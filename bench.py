@@ -101,6 +101,22 @@ def stored_traffic(name: str):
     return None
 
 
+def max_over_ranks(value: float, device, world: int) -> float:
+    """The largest ``value`` over all ranks (the slowest rank's time)."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(bytes_per_step: int, steps: int, ms: float, world: int) -> float:
+    """Whole-job GB/s: every rank's bytes over the slowest rank's interval."""
+    return world * bytes_per_step * steps / (ms * 1e-3) / 1e9
+
+
 # --------------------------------------------------------------------------
 # Clock sampling (NVML, polled during the timed region)
 # --------------------------------------------------------------------------
@@ -281,20 +297,17 @@ def run_ours(args, w, rank: int, world: int, local_rank: int) -> dict | None:
         end.synchronize()
     barrier()
     launches = pqg.pqg_launch_count() - launches0
-    ms = start.elapsed_time(end)
-    if world > 1:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(start.elapsed_time(end), dev, world)
     ms_step = ms / args.steps
     bytes_step = w.algorithmic_bytes()
-    value = world * bytes_step * args.steps / (ms * 1e-3) / 1e9
+    value = job_throughput(bytes_step, args.steps, ms, world)
 
-    # latency at M = 1 (same configuration, one row)
-    lat = latency_m1(w, dev, stream) if rank == 0 else None
-
-    # end to end: pinned host input -> device -> quantize -> codes/scales back
-    e2e = end_to_end(args, w, dev, stream, x0, outs[0], scs[0], mm_ptr, args_c, world)
+    lat = e2e = None
+    if not args.kernel_only:
+        # latency at M = 1 (same configuration, one row)
+        lat = latency_m1(w, dev, stream) if rank == 0 else None
+        # end to end: pinned host input -> device -> quantize -> codes/scales back
+        e2e = end_to_end(args, w, dev, stream, x0, outs[0], scs[0], mm_ptr, args_c, world)
 
     del xs, outs, scs
     torch.cuda.empty_cache()
@@ -325,7 +338,7 @@ def run_ours(args, w, rank: int, world: int, local_rank: int) -> dict | None:
         "gpu_launches": launches,
         "clocks": clocks.summary(),
     }
-    if world == 1 and not args.no_cpu_baseline:
+    if world == 1 and not args.no_cpu_baseline and not args.kernel_only:
         line["cpu_baseline"] = cpu_baseline(w)
     return line
 
@@ -409,12 +422,8 @@ def end_to_end(args, w, dev, stream, x_dev, out_dev, sc_dev, mm_ptr, args_c, wor
         step()
     e1.record(stream)
     e1.synchronize()
-    ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
-    return {"value": world * w.algorithmic_bytes() * steps / (ms * 1e-3) / 1e9, "unit": "GB/s",
+    ms = max_over_ranks(e0.elapsed_time(e1), dev, world)
+    return {"value": job_throughput(w.algorithmic_bytes(), steps, ms, world), "unit": "GB/s",
             "h2d_bytes_per_step": x_host.numel() * x_host.element_size(),
             "d2h_bytes_per_step": out_host.numel() + sc_host.numel(),
             "steps": steps, "ms_per_step": ms / steps}
@@ -428,6 +437,9 @@ def main():
     ap.add_argument("--workload", default="flat_hidden", choices=sorted(workloads()))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--kernel-only", action="store_true",
+                    help="time the kernel loop only (no M=1 latency, e2e or CPU baseline); "
+                         "used for profiler captures")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

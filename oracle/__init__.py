@@ -47,12 +47,19 @@ def build(force: bool = False, src: str = _SRC, out: str = _LIB_PATH) -> str:
 
 
 def load(path: str | None = None):
-    """Load (building first if needed) the oracle library and declare its C API."""
+    """Load (building first if needed) the oracle library and declare its C API.
+
+    ``PQG_ORACLE_LIB`` names another build of ``pqg_oracle.c`` to load instead;
+    the mutation test uses it to run the pins against oracles with planted
+    mistakes."""
     global _lib
-    if path is None and _lib is not None:
+    default = path is None
+    if default and _lib is not None:
         return _lib
+    if default and os.environ.get("PQG_ORACLE_LIB"):
+        path = os.environ["PQG_ORACLE_LIB"]
     with _LOCK:
-        if path is None and _lib is not None:
+        if default and _lib is not None:
             return _lib
         lib = ctypes.CDLL(path or build())
         i64, i32, vp, f32 = ctypes.c_int64, ctypes.c_int, ctypes.c_void_p, ctypes.c_float
@@ -86,7 +93,7 @@ def load(path: str | None = None):
         lib.pqgo_ue8m0_exponent_n.argtypes = [vp, vp, i64]
         lib.pqgo_scale_fp32_n.restype = None
         lib.pqgo_scale_fp32_n.argtypes = [vp, vp, i64, i32]
-        if path is None:
+        if default:
             _lib = lib
         return lib
 

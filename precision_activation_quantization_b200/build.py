@@ -53,9 +53,10 @@ def up_to_date() -> bool:
     return all(os.path.getmtime(d) <= t for d in _inputs())
 
 
-def _compile(src: str, verbose: bool) -> str:
-    obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
-    cmd = [nvcc()] + NVCC_FLAGS + (["-Xptxas", "-v"] if verbose else []) + ["-c", src, "-o", obj]
+def _compile(src: str, verbose: bool, defines=(), build_dir: str = BUILD) -> str:
+    obj = os.path.join(build_dir, os.path.basename(src)[:-3] + ".o")
+    cmd = ([nvcc()] + NVCC_FLAGS + [f"-D{d}" for d in defines]
+           + (["-Xptxas", "-v"] if verbose else []) + ["-c", src, "-o", obj])
     res = subprocess.run(cmd, capture_output=True, text=True)
     if res.returncode != 0:
         raise RuntimeError(f"nvcc failed on {src}:\n{res.stderr}")
@@ -64,20 +65,24 @@ def _compile(src: str, verbose: bool) -> str:
     return obj
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    """Compile and link libpqg.so unless it is newer than every source."""
-    if not force and up_to_date():
+def build(force: bool = False, verbose: bool = False, defines=(), out: str = LIB) -> str:
+    """Compile and link libpqg.so unless it is newer than every source.
+
+    ``defines`` (e.g. ``["PQG_ITEMS_PLAIN=4"]``) set the build-time tuning
+    macros; with ``out`` they build a variant library elsewhere."""
+    if not force and not defines and out == LIB and up_to_date():
         return LIB
-    os.makedirs(BUILD, exist_ok=True)
+    build_dir = BUILD if not defines else os.path.join(BUILD, "_".join(defines).replace("=", ""))
+    os.makedirs(build_dir, exist_ok=True)
     with cf.ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 1)) as ex:
-        objs = list(ex.map(lambda s: _compile(s, verbose), sources()))
-    tmp = LIB + f".tmp{os.getpid()}"
+        objs = list(ex.map(lambda s: _compile(s, verbose, defines, build_dir), sources()))
+    tmp = out + f".tmp{os.getpid()}"
     cmd = [nvcc()] + ARCH + ["-shared", "-cudart", "static", "-o", tmp] + objs
     res = subprocess.run(cmd, capture_output=True, text=True)
     if res.returncode != 0:
         raise RuntimeError(f"link failed:\n{res.stderr}")
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, out)
+    return out
 
 
 def main() -> None:

@@ -26,10 +26,17 @@ struct LaunchArgs {
 
 int sm_count(int device);  // cached cudaDevAttrMultiProcessorCount
 
-// Strips each warp takes per iteration (loads in flight per lane).
+// Strips each warp takes per iteration: each lane keeps this many 32-byte
+// loads in flight (twice as many when fused).  Tunable at build time.
+#ifndef PQG_ITEMS_PLAIN
+#define PQG_ITEMS_PLAIN 2
+#endif
+#ifndef PQG_ITEMS_FUSED
+#define PQG_ITEMS_FUSED 2
+#endif
 template <bool FUSED>
 constexpr int items_per_warp() {
-    return FUSED ? 2 : 2;
+    return FUSED ? PQG_ITEMS_FUSED : PQG_ITEMS_PLAIN;
 }
 
 template <typename In, int G, Kind KIND, bool FUSED>

@@ -108,10 +108,11 @@ def _scale_planes(w, sbytes):
 
 
 def check_fused(w, *, max_flip_frac=1e-4, rel_tol=7e-2, **kw):
-    """Fused contract: scales equal (fp32 within 1 ulp; UE8M0 equal unless the
-    oracle's amax/448 is within 2^-20 of a power of two); codes equal except for
-    at most ``max_flip_frac`` of elements that move by one step; every element's
-    dequantized value within ``rel_tol`` of the oracle's silu(gate)*up."""
+    """Fused contract: UE8M0 bytes equal unless the oracle's amax/448 is within
+    2^-20 of a power of two; fp32 scales within 2^-19 relative; codes equal
+    except for at most ``max_flip_frac`` of elements (outside groups whose UE8M0
+    exponent flipped), each moving by one step; every element's dequantized
+    value within ``rel_tol`` of the oracle's silu(gate)*up."""
     gq, gs = run_gpu(w, **kw)
     rq, rs = run_oracle(w)
     E, M, K, G = w.E, w.M, w.K, w.group
@@ -157,16 +158,19 @@ def check_fused(w, *, max_flip_frac=1e-4, rel_tol=7e-2, **kw):
         near_pow2 = np.abs(r / np.exp2(np.round(np.log2(r))) - 1.0) < 2.0 ** -20
         assert (~scale_diff | near_pow2).all(), \
             f"{w.name}: {int((scale_diff & ~near_pow2).sum())} UE8M0 bytes differ away from a power of two"
+        exempt = scale_diff            # an exponent flip rescales the whole group
     else:
-        ulps = np.abs(g_sc.astype(np.float32).view(np.int32).astype(np.int64)
-                      - r_sc.astype(np.float32).view(np.int32).astype(np.int64))
-        assert ulps.max(initial=0) <= 1, f"{w.name}: fp32 scale off by {ulps.max()} ulp"
-        scale_diff = ulps > 0
+        # the device forms silu(gate)*up in fp32 (a few ulps from the oracle's
+        # double), so the group absmax, and with it the scale, may move by a
+        # few ulps: bound it at 2^-19 relative
+        rel = np.abs(g_sc / r_sc - 1.0)
+        assert rel.max(initial=0) <= 2.0 ** -19, f"{w.name}: fp32 scale off by {rel.max():.3g}"
+        exempt = np.zeros_like(g_sc, dtype=bool)
+        scale_diff = rel > 0
 
     gcodes = gq3[live].reshape(-1, K // G, G)
     rcodes = rq3[live].reshape(-1, K // G, G)
-    same_scale = ~scale_diff
-    diff = (gcodes != rcodes) & same_scale[..., None]
+    diff = (gcodes != rcodes) & ~exempt[..., None]
     n_el = gcodes.size
     if w.out_dtype == "int8":
         step = np.abs(gcodes.view(np.int8).astype(np.int64) - rcodes.view(np.int8).astype(np.int64))

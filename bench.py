@@ -49,6 +49,8 @@ def workloads():
     return {
         "flat_hidden": lambda: inputs.flat_hidden(),
         "flat_hidden_fp32": lambda: inputs.flat_hidden(layout="row", scale_fmt="fp32"),
+        "per_token": lambda: inputs.flat_hidden(layout="row", scale_fmt="fp32").with_(
+            group=7168, name="per_token_8192x7168"),
         "fused": lambda: inputs.fused(),
         "masked": lambda: inputs.masked(),
         "masked_decode": lambda: inputs.masked(decode=True),
@@ -284,19 +286,37 @@ def run_ours(args, w, rank: int, world: int, local_rank: int) -> dict | None:
             dist.barrier()
         torch.cuda.synchronize(dev)
 
+    graph = None
+    if args.graph:
+        # the K timed steps captured once as a CUDA graph (host launch cost out
+        # of the timed region); warm-up steps run eagerly before capture
+        stream = torch.cuda.Stream(dev)
+        sh = stream.cuda_stream
     for i in range(args.warmup):
         launch(i)
+    if args.graph:
+        torch.cuda.synchronize(dev)
+        graph = torch.cuda.CUDAGraph()
+        captured0 = pqg.pqg_launch_count()
+        with torch.cuda.graph(graph, stream=stream):
+            for i in range(args.steps):
+                launch(args.warmup + i)
+        captured = pqg.pqg_launch_count() - captured0
     barrier()
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     launches0 = pqg.pqg_launch_count()
     with ClockSampler(dev.index) as clocks:
         start.record(stream)
-        for i in range(args.steps):
-            launch(args.warmup + i)
+        if graph is not None:
+            graph.replay()
+        else:
+            for i in range(args.steps):
+                launch(args.warmup + i)
         end.record(stream)
         end.synchronize()
     barrier()
-    launches = pqg.pqg_launch_count() - launches0
+    launches = captured if graph is not None else pqg.pqg_launch_count() - launches0
+    del graph
     ms = max_over_ranks(start.elapsed_time(end), dev, world)
     ms_step = ms / args.steps
     bytes_step = w.algorithmic_bytes()
@@ -322,7 +342,8 @@ def run_ours(args, w, rank: int, world: int, local_rank: int) -> dict | None:
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic",
-        "config": dict(describe(w), l2=f"{sets} rotating buffer sets ({sets * footprint / 1e6:.0f} MB "
+        "config": dict(describe(w), launch="cuda-graph replay" if args.graph else "stream",
+                       l2=f"{sets} rotating buffer sets ({sets * footprint / 1e6:.0f} MB "
                                        f"> 4 x 126 MB L2); each step reads a set last used "
                                        f"{sets - 1} steps earlier",
                        parallelism=f"{world} independent replica(s), no data-path collective"),
@@ -437,6 +458,8 @@ def main():
     ap.add_argument("--workload", default="flat_hidden", choices=sorted(workloads()))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--graph", action="store_true",
+                    help="replay the K timed steps from one CUDA graph (launch-bound workloads)")
     ap.add_argument("--kernel-only", action="store_true",
                     help="time the kernel loop only (no M=1 latency, e2e or CPU baseline); "
                          "used for profiler captures")

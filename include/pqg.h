@@ -121,10 +121,12 @@ enum pqg_scale_layout {
  *          scales and packed words, any alignment for UE8M0 bytes.
  * M        rows per expert (with masked_m: the capacity M_max of each expert).
  *          M >= 0; M == 0 launches nothing.
- * num_experts  >= 1 (<= 65535).  With masked_m == NULL every expert's M rows
+ * num_experts  1 ..= 4096.  With masked_m == NULL every expert's M rows
  *          are quantized (num_experts == 1 is the flat dispatch).
  * K        output elements per row, a positive multiple of group.
- * group    G in {32, 64, 128}.
+ * group    G in {32, 64, 128}, or G == K for one scale per row (per-token
+ *          quantization, as tf_per_token_quant_fp8 on the TeleFuser page;
+ *          K a multiple of 16, at most 16384).
  * in_dtype PQG_BF16 or PQG_FP16.   out_dtype PQG_E4M3 or PQG_INT8.
  * scale_fmt, scale_layout   see above.  PQG_SCALE_UE8M0 requires PQG_E4M3, and
  *          PQG_UE8M0_PACKED requires PQG_SCALE_UE8M0 (else PQG_ERR_UNSUPPORTED).
@@ -141,8 +143,8 @@ enum pqg_scale_layout {
  *          waits for the preceding grid before its first global-memory access.
  *
  * Returns PQG_OK, or a negative pqg_status with nothing launched (except
- * PQG_ERR_CUDA).  Limits: K <= 2^28, M * ceil(K / 512) < 2^31 and
- * num_experts * M * K <= 2^40 (else PQG_ERR_INVALID_ARG).
+ * PQG_ERR_CUDA).  Limits: K <= 2^28, num_experts * M * ceil(K / 512) < 2^31
+ * and num_experts * M * K <= 2^40 (else PQG_ERR_INVALID_ARG).
  * The output and scale buffers must not overlap the input.
  */
 PQG_API int pqg_quant(const void *in, void *out, void *scales, int64_t M,

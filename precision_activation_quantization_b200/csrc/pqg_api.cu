@@ -21,8 +21,9 @@ std::atomic<uint64_t> g_launches{0};
 
 constexpr int64_t kMaxDevices = 64;
 std::atomic<int> g_sm_count[kMaxDevices];
-
 int64_t padded_rows(int64_t M) { return (M + 3) / 4 * 4; }
+
+constexpr int64_t kMaxPerTokenK = 16384;
 
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
@@ -35,16 +36,19 @@ int check_geometry(int64_t num_experts, int64_t M, int64_t K, int group, int sca
         scale_layout != PQG_UE8M0_PACKED)
         return PQG_ERR_INVALID_ARG;
     if (group <= 0) return PQG_ERR_INVALID_ARG;
-    if (group != 32 && group != 64 && group != 128) return PQG_ERR_UNSUPPORTED;
+    // G in {32, 64, 128}, or one group per row (per-token, K <= 16384)
+    const bool per_token = group == K && K % 16 == 0 && K <= kMaxPerTokenK;
+    if (group != 32 && group != 64 && group != 128 && !per_token) return PQG_ERR_UNSUPPORTED;
     if (scale_layout == PQG_UE8M0_PACKED && scale_fmt != PQG_SCALE_UE8M0)
         return PQG_ERR_UNSUPPORTED;
-    if (num_experts < 1 || num_experts > 65535) return PQG_ERR_INVALID_ARG;
+    if (num_experts < 1 || num_experts > static_cast<int64_t>(pqg::kMaxExperts))
+        return PQG_ERR_INVALID_ARG;
     if (M < 0 || K <= 0 || K % group != 0) return PQG_ERR_INVALID_ARG;
     // 2K-byte (4K fused) rows must fit the 32-bit row stride; strips per expert
     // must fit a 32-bit index.
     if (K > (int64_t{1} << 28)) return PQG_ERR_INVALID_ARG;
     const int64_t segs = (K + pqg::kStripElems - 1) / pqg::kStripElems;
-    if (M > 0 && M >= (int64_t{1} << 31) / segs) return PQG_ERR_INVALID_ARG;
+    if (M > 0 && M >= (int64_t{1} << 31) / (segs * num_experts)) return PQG_ERR_INVALID_ARG;
     if (M * K > (int64_t{1} << 40) / num_experts) return PQG_ERR_INVALID_ARG;
 
     const int64_t ng = K / group;
@@ -130,9 +134,11 @@ int pqg_quant(const void *in, void *out, void *scales, int64_t M, int64_t num_ex
     a.p.segs = static_cast<uint32_t>((K + pqg::kStripElems - 1) / pqg::kStripElems);
     a.p.mpad = static_cast<uint32_t>(padded_rows(M));
     a.p.layout = static_cast<uint32_t>(scale_layout);
-    a.experts = static_cast<uint32_t>(num_experts);
-    a.grid_rows = static_cast<uint32_t>(
-        (masked_m != nullptr && expected_m > 0 && expected_m < M) ? expected_m : M);
+    a.p.experts = static_cast<uint32_t>(num_experts);
+    const int64_t grid_rows =
+        (masked_m != nullptr && expected_m > 0 && expected_m < M) ? expected_m : M;
+    a.expected_strips = static_cast<uint64_t>(num_experts * grid_rows) * a.p.segs;
+    a.expected_rows = static_cast<uint64_t>(num_experts * grid_rows);
     a.group = group;
     a.kind = scale_fmt == PQG_SCALE_UE8M0 ? pqg::Kind::E4M3_UE8M0
              : out_dtype == PQG_INT8      ? pqg::Kind::INT8_FP32

@@ -11,12 +11,19 @@
 //
 // Work decomposition.  A "strip" is 32 lanes x 16 elements = 512 consecutive
 // outputs of one row, so each lane owns 16 outputs (32 bytes of bf16/fp16
-// input, read with one 256-bit load; the report's 执行摘要 names the same 32 B
-// per lane tiling).  A 1 x G group spans L = G/16 adjacent lanes; its absmax is
-// a log2(L)-step xor-shuffle.  Each warp takes ITEMS consecutive strips per
-// iteration and issues all their loads before any arithmetic, so every lane has
-// ITEMS (x2 when fused) independent 32-byte loads in flight.  Rows whose width
-// is not a multiple of 512 leave the tail lanes of their last strip idle.
+// input, one 256-bit load; the report's 执行摘要 names the same 32 B per lane
+// tiling).  A 1 x G group spans L = G/16 adjacent lanes; its absmax is a
+// log2(L)-step xor-shuffle.  The strips of all experts (rows < masked_m[e]
+// only) form one sequence, cut into blocks of WARPS x ITEMS strips that the
+// CTAs take round-robin.  With several experts each CTA first prefix-sums the
+// per-expert strip counts in shared memory, so a warp can find the expert and
+// row of any strip; skewed masked_m cannot leave CTAs idle.
+//
+// Memory-level parallelism.  A warp takes ITEMS strips per chunk and issues
+// all of the chunk's 32-byte loads before any arithmetic; with about 40
+// resident warps per SM (register-light kernel) that keeps the HBM queues full.
+// Keeping a second chunk in flight (register double-buffering) was measured
+// slower: the extra registers cost more warps than the prefetch won.
 //
 // Exact division.  Codes must equal a rounding of fp32(x / s).  A per-element
 // IEEE division is too slow for a bandwidth-bound loop, so the quotient is
@@ -29,6 +36,12 @@
 // but every such t rounds to a signed zero code, and the sign is restored from
 // x.  The correction runs on packed f32x2 FMAs (FFMA2), two elements per
 // instruction.
+//
+// UE8M0 exponent without a division.  For a normal fp32 amax = m * 2^E (m in
+// [1, 2)), the smallest n with 448 * 2^n >= amax is E - 8 + [m > 1.75], because
+// 448 = 1.75 * 2^8.  The pages' rule (biased exponent of fp32(amax/448), plus
+// one for a nonzero mantissa) gives the same byte for every fp32 amax >= 1e-10:
+// an exhaustive check over all 1.35e9 such values found no difference.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -36,6 +49,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <type_traits>
 
 namespace pqg {
 
@@ -44,15 +58,15 @@ enum class Kind : int { E4M3_FP32 = 0, E4M3_UE8M0 = 1, INT8_FP32 = 2 };
 // Runtime scale layouts (same numbering as the C ABI's pqg_scale_layout).
 enum : uint32_t { kRowMajor = 0, kColMajor = 1, kPacked = 2 };
 
-constexpr int kWarps = 8;                  // warps per CTA
-constexpr int kThreads = kWarps * 32;
 constexpr int kStripElems = 512;           // outputs per strip (32 lanes x 16)
+constexpr uint32_t kStripBytes = 1024;     // input bytes per strip (16-bit elements)
+constexpr uint32_t kMaxExperts = 4096;     // prefix table lives in shared memory
 
 struct Params {
     const uint8_t *in;         // expert 0, row 0
     uint8_t *out;              // expert 0, row 0
     uint8_t *scales;           // expert 0's scale plane (byte address)
-    const int32_t *masked_m;   // device int32[E], or null: all M rows
+    const int32_t *masked_m;   // device int32[experts], or null: all M rows
     int64_t in_expert_bytes;   // M * in_row_bytes
     int64_t out_expert_bytes;  // M * K
     int64_t scale_expert_bytes;
@@ -63,7 +77,15 @@ struct Params {
     uint32_t segs;             // strips per row = ceil(K / 512)
     uint32_t mpad;             // rows of a column-major plane (M rounded up to 4)
     uint32_t layout;           // kRowMajor / kColMajor / kPacked
+    uint32_t experts;          // <= kMaxExperts
+    uint32_t items;            // strips per warp per block, 1 .. ITEMS
 };
+
+// Dynamic shared memory of one CTA: the expert prefix table (more than 32
+// experts only).
+__host__ __device__ constexpr uint32_t smem_bytes(uint32_t experts) {
+    return experts > 32u ? 4u * (experts + 1u) : 0u;
+}
 
 // ---------------------------------------------------------------------------
 // Memory helpers
@@ -149,14 +171,65 @@ __device__ __forceinline__ float2 div_rn2(float2 x, float2 y, float2 ns) {
     return q;
 }
 
-// t keeps the sign of x: differs from q only when q is a zero of the wrong sign.
-__device__ __forceinline__ float with_sign_of(float q, float x) {
-    return __uint_as_float(__float_as_uint(q) | (__float_as_uint(x) & 0x80000000u));
+// The same correction carried on the negated quotient, from ny = -RN(1/s) and
+// s: returns -RN(x/s) with the sign of zero right for every x.  (q = x*ny and
+// r = x + q*s: for x = -0 the chain gives +0, for x = +0 it gives -0, and a
+// tiny x whose quotient underflows keeps the sign of -x.)  Negating the codes
+// afterwards is one XOR of the packed sign bits.
+__device__ __forceinline__ float2 neg_div_rn2(float2 x, float2 ny, float2 s) {
+    float2 q = __fmul2_rn(x, ny);
+    float2 r = __ffma2_rn(q, s, x);    // x - (x/s)*s, exact
+    q = __ffma2_rn(r, ny, q);
+    r = __ffma2_rn(q, s, x);
+    q = __ffma2_rn(r, ny, q);
+    return q;
+}
+
+// bf16 x * 2^k with an exact bf16 power of two, widened: one mixed-precision
+// FMA (bf16 x bf16 + f32 -> f32).  Adding -0 keeps every product, -0 included.
+__device__ __forceinline__ float mul_bf16_pow2(uint16_t x, uint16_t p2) {
+    float d;
+    asm("fma.rn.f32.bf16 %0, %1, %2, %3;" : "=f"(d) : "h"(x), "h"(p2), "f"(-0.0f));
+    return d;
+}
+
+// max |x| over the 16 bf16/fp16 values of 8 packed words, as the 16-bit
+// pattern of the largest magnitude (finite values order like their magnitude
+// bits).
+__device__ __forceinline__ uint32_t absmax_bits16(const uint32_t (&w)[8]) {
+    uint32_t m[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) m[i] = w[i] & 0x7FFF7FFFu;
+    uint32_t a = __vimax3_u16x2(m[0], m[1], m[2]);
+    uint32_t b = __vimax3_u16x2(m[3], m[4], m[5]);
+    a = __vimax3_u16x2(a, b, __vimax3_u16x2(m[6], m[7], 0u));
+    return max(a & 0xFFFFu, a >> 16);
 }
 
 // ---------------------------------------------------------------------------
 // Per-group scale math (one group per L lanes; all lanes compute it)
 // ---------------------------------------------------------------------------
+
+// UE8M0 byte of a (normal, >= 1e-10) amax: E(amax) - 8 + [mantissa > 0x600000],
+// i.e. 127 + ceil(log2(amax / 448)); see the file comment.
+__device__ __forceinline__ uint32_t ue8m0_exponent(float amax) {
+    const uint32_t b = __float_as_uint(amax);
+    return ((b >> 23) & 0xFFu) - 8u + ((b & 0x7FFFFFu) > 0x600000u ? 1u : 0u);
+}
+
+// RN(a / c) for the scale divisors: q = a * RN(1/c), then two Markstein
+// corrections with exact FMA residuals.  An exhaustive CPU check over every
+// fp32 a >= 1e-10 (1.35e9 values) found it equal to the IEEE quotient for both
+// c = 448 and c = 127.
+constexpr float kRcp448 = 0x1.24924ap-9f;   // RN(1/448)
+constexpr float kRcp127 = 0x1.020408p-7f;   // RN(1/127)
+__device__ __forceinline__ float div_by_const(float a, float c, float rc) {
+    float q = __fmul_rn(a, rc);
+    float r = __fmaf_rn(-q, c, a);
+    q = __fmaf_rn(r, rc, q);
+    r = __fmaf_rn(-q, c, a);
+    return __fmaf_rn(r, rc, q);
+}
 
 struct GroupScale {
     float mult;   // UE8M0: 2^(127-e) (exact); fp32 kinds: y = RN(1/s)
@@ -170,14 +243,13 @@ __device__ __forceinline__ GroupScale make_scale(float amax) {
     GroupScale gs;
     amax = fmaxf(amax, 1e-10f);   // EPS floor
     if constexpr (KIND == Kind::E4M3_UE8M0) {
-        const float raw = __fdiv_rn(amax, 448.0f);
-        const uint32_t b = __float_as_uint(raw);
-        gs.e8 = ((b >> 23) & 0xFFu) + ((b & 0x7FFFFFu) != 0u);
+        gs.e8 = ue8m0_exponent(amax);
         gs.mult = __uint_as_float((254u - gs.e8) << 23);
         gs.s = 0.0f;
         gs.neg_s = 0.0f;
     } else {
-        gs.s = __fdiv_rn(amax, KIND == Kind::INT8_FP32 ? 127.0f : 448.0f);
+        gs.s = KIND == Kind::INT8_FP32 ? div_by_const(amax, 127.0f, kRcp127)
+                                       : div_by_const(amax, 448.0f, kRcp448);
         gs.mult = __frcp_rn(gs.s);
         gs.neg_s = -gs.s;
         gs.e8 = 0;
@@ -199,16 +271,14 @@ __device__ __forceinline__ void encode16(const float (&v)[16], const GroupScale 
             w[j] = e4m3x2(a.x, a.y) | (e4m3x2(b.x, b.y) << 16);
         }
     } else if constexpr (KIND == Kind::E4M3_FP32) {
-        const float2 y2 = make_float2(gs.mult, gs.mult);
-        const float2 ns2 = make_float2(gs.neg_s, gs.neg_s);
+        // codes of -t, then the four sign bits flipped at once
+        const float2 ny2 = make_float2(-gs.mult, -gs.mult);
+        const float2 s2 = make_float2(gs.s, gs.s);
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-            float2 xa = make_float2(v[4 * j], v[4 * j + 1]);
-            float2 xb = make_float2(v[4 * j + 2], v[4 * j + 3]);
-            float2 a = div_rn2(xa, y2, ns2);
-            float2 b = div_rn2(xb, y2, ns2);
-            w[j] = e4m3x2(with_sign_of(a.x, xa.x), with_sign_of(a.y, xa.y)) |
-                   (e4m3x2(with_sign_of(b.x, xb.x), with_sign_of(b.y, xb.y)) << 16);
+            const float2 a = neg_div_rn2(make_float2(v[4 * j], v[4 * j + 1]), ny2, s2);
+            const float2 b = neg_div_rn2(make_float2(v[4 * j + 2], v[4 * j + 3]), ny2, s2);
+            w[j] = (e4m3x2(a.x, a.y) | (e4m3x2(b.x, b.y) << 16)) ^ 0x80808080u;
         }
     } else {
         // INT8: adding 1.5 * 2^23 rounds |t| < 2^22 to an integer (ties to even)
@@ -230,128 +300,327 @@ __device__ __forceinline__ void encode16(const float (&v)[16], const GroupScale 
 }
 
 // ---------------------------------------------------------------------------
+// The strip sequence: which expert, row and strip-in-row a strip index is
+// ---------------------------------------------------------------------------
+//
+// Strips of expert e are [start_e, start_e + strips_e); strips_e =
+// rows_e * segs with rows_e = clamp(masked_m[e], 0, M) (M without masked_m).
+// Three representations, picked per launch:
+//   one expert   : start 0, strips = total (no table at all);
+//   <= 32 experts: a warp-register table, lane e holding expert e's count and
+//                  inclusive prefix; a lookup is one ballot and two shuffles;
+//   more experts : a shared-memory prefix table built by the CTA.
+
+constexpr uint32_t kWarpTableExperts = 32;
+
+struct ExpertTable {
+    uint32_t mode;     // 0 one expert, 1 warp table, 2 shared-memory table
+    uint32_t total;    // strips of all experts
+    uint32_t incl;     // mode 1: this lane's inclusive prefix (total for lanes >= E)
+    uint32_t cnt;      // mode 1: this lane's expert's strips
+    const uint32_t *prefix;  // mode 2: prefix[e] = start_e, prefix[E] = total
+};
+
+struct Span {
+    uint32_t e, start, strips;
+};
+
+__device__ __forceinline__ uint32_t expert_strips(const Params &p, uint32_t e) {
+    uint32_t rows = p.M;
+    if (p.masked_m != nullptr) {
+        const int mm = __ldg(p.masked_m + e);
+        rows = static_cast<uint32_t>(min(max(mm, 0), static_cast<int>(p.M)));
+    }
+    return rows * p.segs;
+}
+
+// prefix[e] = strips of experts 0..e-1.  Every thread of the CTA calls it; it
+// ends with __syncthreads.
+__device__ __forceinline__ void build_prefix(const Params &p, uint32_t *prefix) {
+    __shared__ uint32_t warp_sums[32];
+    const uint32_t n = blockDim.x, t = threadIdx.x, lane = t & 31u, warp = t >> 5;
+    const uint32_t per = (p.experts + n - 1) / n;
+    const uint32_t lo = min(t * per, p.experts), hi = min(lo + per, p.experts);
+    uint32_t local = 0;
+    for (uint32_t e = lo; e < hi; ++e) local += expert_strips(p, e);
+    uint32_t incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+        if (lane >= static_cast<uint32_t>(o)) incl += v;
+    }
+    if (lane == 31) warp_sums[warp] = incl;
+    __syncthreads();
+    uint32_t base = 0;
+    for (uint32_t w = 0; w < warp; ++w) base += warp_sums[w];
+    uint32_t run = base + incl - local;
+    for (uint32_t e = lo; e < hi; ++e) {
+        prefix[e] = run;
+        run += expert_strips(p, e);
+    }
+    if (t == n - 1) prefix[p.experts] = base + incl;
+    __syncthreads();
+}
+
+// Build the table (every thread of the CTA calls it).
+__device__ __forceinline__ ExpertTable make_table(const Params &p, uint32_t *smem_prefix,
+                                                  uint32_t lane) {
+    ExpertTable t;
+    t.incl = t.cnt = 0;
+    t.prefix = smem_prefix;
+    if (p.experts == 1) {
+        t.mode = 0;
+        t.total = expert_strips(p, 0);
+    } else if (p.experts <= kWarpTableExperts) {
+        t.mode = 1;
+        t.cnt = lane < p.experts ? expert_strips(p, lane) : 0u;
+        uint32_t incl = t.cnt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+            if (lane >= static_cast<uint32_t>(o)) incl += v;
+        }
+        t.incl = incl;
+        t.total = __shfl_sync(0xFFFFFFFFu, incl, 31);
+    } else {
+        t.mode = 2;
+        build_prefix(p, smem_prefix);
+        t.total = smem_prefix[p.experts];
+    }
+    return t;
+}
+
+// The expert holding strip s (s < total).  Warp-uniform s; every lane calls.
+__device__ __forceinline__ Span locate(const ExpertTable &t, uint32_t experts, uint32_t s) {
+    Span sp;
+    if (t.mode == 0) {
+        sp.e = 0;
+        sp.start = 0;
+        sp.strips = t.total;
+    } else if (t.mode == 1) {
+        // experts whose whole range lies at or below s come first
+        sp.e = __popc(__ballot_sync(0xFFFFFFFFu, t.incl <= s));
+        const uint32_t incl = __shfl_sync(0xFFFFFFFFu, t.incl, sp.e);
+        sp.strips = __shfl_sync(0xFFFFFFFFu, t.cnt, sp.e);
+        sp.start = incl - sp.strips;
+    } else {
+        uint32_t lo = 0, hi = experts;  // prefix[lo] <= s < prefix[hi]
+        while (hi - lo > 1) {
+            const uint32_t mid = (lo + hi) >> 1;
+            if (t.prefix[mid] <= s) lo = mid; else hi = mid;
+        }
+        sp.e = lo;
+        sp.start = t.prefix[lo];
+        sp.strips = t.prefix[lo + 1] - sp.start;
+    }
+    return sp;
+}
+
+// ---------------------------------------------------------------------------
+// One chunk of up to ITEMS strips held in registers
+// ---------------------------------------------------------------------------
+
+template <int ITEMS, bool FUSED>
+struct Chunk {
+    uint32_t x[ITEMS][8];              // raw 16-bit pairs (gate when fused)
+    uint32_t u[ITEMS][FUSED ? 8 : 1];  // up half when fused
+    uint32_t e[ITEMS], row[ITEMS], col[ITEMS];
+    uint32_t n;                        // strips in this chunk (warp-uniform)
+};
+
+// Issue the loads of strips [s, s + n) (n <= ITEMS).  Lanes past the end of a
+// ragged row load nothing.  With one expert (MULTI false) the strip index maps
+// to (row, strip-in-row) by one division; otherwise through the expert table.
+template <int ITEMS, bool FUSED, bool MULTI>
+__device__ __forceinline__ void load_chunk(Chunk<ITEMS, FUSED> &ch, uint32_t s, uint32_t n,
+                                           const ExpertTable &t, const Params &p,
+                                           uint32_t lane) {
+    ch.n = n;
+    uint32_t e = 0, start = 0, end_e = t.total;
+    if constexpr (MULTI) {
+        const Span sp = locate(t, p.experts, s);
+        e = sp.e;
+        start = sp.start;
+        end_e = sp.start + sp.strips;
+    }
+    uint32_t row = (s - start) / p.segs;
+    uint32_t seg = (s - start) - row * p.segs;
+#pragma unroll
+    for (int k = 0; k < ITEMS; ++k) {
+        const bool live = static_cast<uint32_t>(k) < n;
+        if constexpr (MULTI) {
+            if (live && s + k >= end_e) {        // the chunk runs into the next expert
+                const Span sp = locate(t, p.experts, s + k);
+                e = sp.e;
+                start = sp.start;
+                end_e = sp.start + sp.strips;
+                row = 0;
+                seg = 0;
+            }
+        }
+        ch.e[k] = e;
+        ch.row[k] = row;
+        ch.col[k] = seg * kStripElems + lane * 16u;
+        if (live && ch.col[k] < p.K) {
+            const uint8_t *src = p.in + e * p.in_expert_bytes +
+                                 static_cast<uint64_t>(row) * p.in_row_bytes +
+                                 static_cast<uint64_t>(ch.col[k]) * 2u;
+            load32B(src, ch.x[k]);
+            if constexpr (FUSED) load32B(src + static_cast<uint64_t>(p.K) * 2u, ch.u[k]);
+        } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                ch.x[k][i] = 0u;
+                if constexpr (FUSED) ch.u[k][i] = 0u;
+            }
+        }
+        if (++seg == p.segs) {
+            seg = 0;
+            ++row;
+        }
+    }
+}
+
+// bf16 UE8M0 through the mixed-precision FMA path (1) or by widening (0).
+#ifndef PQG_UE8M0_MIXED
+#define PQG_UE8M0_MIXED 1
+#endif
+
+// Quantize one strip held in registers and store its codes and scales.
+template <typename In, int G, Kind KIND, bool FUSED>
+__device__ __forceinline__ void quantize_strip(const uint32_t (&x)[8], const uint32_t *u,
+                                               uint32_t e, uint32_t row, uint32_t col,
+                                               const Params &p, uint32_t lane) {
+    constexpr int L = G / 16;  // lanes per group
+    const bool ok = col < p.K;
+    const uint32_t g = col / G;  // group within the row (valid lanes)
+    const uint32_t sub = lane % L;
+    uint32_t w[4];
+    GroupScale gs;
+
+    constexpr bool kMixed = PQG_UE8M0_MIXED && KIND == Kind::E4M3_UE8M0 && !FUSED &&
+                            std::is_same<In, __nv_bfloat16>::value;
+    if constexpr (kMixed) {
+        // absmax on the raw bits, t = x * 2^k by a mixed bf16 FMA: no widening
+        uint32_t ab = absmax_bits16(x);
+#pragma unroll
+        for (int o = 1; o < L; o <<= 1) ab = max(ab, __shfl_xor_sync(0xFFFFFFFFu, ab, o));
+        gs.e8 = ue8m0_exponent(fmaxf(__uint_as_float(ab << 16), 1e-10f));
+        const uint16_t p2 = static_cast<uint16_t>((254u - gs.e8) << 7);  // bf16 2^(127-e)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const uint32_t a = x[2 * j], b = x[2 * j + 1];
+            const float t0 = mul_bf16_pow2(static_cast<uint16_t>(a & 0xFFFFu), p2);
+            const float t1 = mul_bf16_pow2(static_cast<uint16_t>(a >> 16), p2);
+            const float t2 = mul_bf16_pow2(static_cast<uint16_t>(b & 0xFFFFu), p2);
+            const float t3 = mul_bf16_pow2(static_cast<uint16_t>(b >> 16), p2);
+            w[j] = e4m3x2(t0, t1) | (e4m3x2(t2, t3) << 16);
+        }
+    } else {
+        float v[16];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            widen2<In>(x[i], v[2 * i], v[2 * i + 1]);
+            if constexpr (FUSED) {
+                float u0, u1;
+                widen2<In>(u[i], u0, u1);
+                v[2 * i] = silu_mul(v[2 * i], u0);
+                v[2 * i + 1] = silu_mul(v[2 * i + 1], u1);
+            }
+        }
+        float amax = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
+#pragma unroll
+        for (int o = 1; o < L; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+        gs = make_scale<KIND>(amax);
+        encode16<KIND>(v, gs, w);
+    }
+
+    uint32_t packed_word = 0;
+    if constexpr (KIND == Kind::E4M3_UE8M0) {
+        // little-endian word of groups 4j..4j+3 assembled across the 4 groups'
+        // lanes (invalid groups contribute 0)
+        packed_word = ok ? (gs.e8 << (8u * (g & 3u))) : 0u;
+        packed_word |= __shfl_xor_sync(0xFFFFFFFFu, packed_word, L);
+        packed_word |= __shfl_xor_sync(0xFFFFFFFFu, packed_word, 2 * L);
+    }
+    if (!ok) return;
+
+    store16B(p.out + e * p.out_expert_bytes + static_cast<uint64_t>(row) * p.K + col, w[0], w[1],
+             w[2], w[3]);
+    if (sub == 0) {
+        uint8_t *sc = p.scales + e * p.scale_expert_bytes;
+        if (p.layout == kPacked) {
+            if ((g & 3u) == 0u)
+                reinterpret_cast<uint32_t *>(sc)[static_cast<uint64_t>(g >> 2) * p.mpad + row] =
+                    packed_word;
+        } else {
+            const uint64_t idx = (p.layout == kRowMajor) ? static_cast<uint64_t>(row) * p.ng + g
+                                                         : static_cast<uint64_t>(g) * p.mpad + row;
+            if constexpr (KIND == Kind::E4M3_UE8M0)
+                sc[idx] = static_cast<uint8_t>(gs.e8);
+            else
+                reinterpret_cast<float *>(sc)[idx] = gs.s;
+        }
+    }
+}
+
+template <typename In, int G, Kind KIND, bool FUSED, int ITEMS>
+__device__ __forceinline__ void quantize_chunk(const Chunk<ITEMS, FUSED> &ch, const Params &p,
+                                               uint32_t lane) {
+#pragma unroll
+    for (int k = 0; k < ITEMS; ++k) {
+        if (static_cast<uint32_t>(k) >= ch.n) break;  // warp-uniform
+        quantize_strip<In, G, KIND, FUSED>(ch.x[k], FUSED ? ch.u[k] : nullptr, ch.e[k],
+                                           ch.row[k], ch.col[k], p, lane);
+    }
+}
+
+// ---------------------------------------------------------------------------
 // The kernel
 // ---------------------------------------------------------------------------
 
-template <typename In, int G, Kind KIND, bool FUSED, int ITEMS>
-__global__ void __launch_bounds__(kThreads) quant_kernel(const __grid_constant__ Params p) {
-    constexpr int L = G / 16;                   // lanes per group
-    static_assert(L >= 2 && L <= 8 && (L & (L - 1)) == 0, "G must be 32, 64 or 128");
+// Resident CTAs per SM the register allocation must allow (0: no constraint).
+// The fp32-scale plain variants run best at 5 (<= 51 registers); the rest need
+// no constraint.
+#ifndef PQG_MIN_BLOCKS_FP32
+#define PQG_MIN_BLOCKS_FP32 5
+#endif
+template <Kind KIND, bool FUSED>
+constexpr int min_blocks() {
+    return (KIND != Kind::E4M3_UE8M0 && !FUSED) ? PQG_MIN_BLOCKS_FP32 : 0;
+}
 
-    wait_for_producer();
+template <typename In, int G, Kind KIND, bool FUSED, int ITEMS, int WARPS, bool MULTI>
+__global__ void __launch_bounds__(WARPS * 32, min_blocks<KIND, FUSED>())
+    quant_kernel(const __grid_constant__ Params p) {
+    static_assert(G == 32 || G == 64 || G == 128, "G must be 32, 64 or 128");
+    extern __shared__ __align__(16) uint32_t smem_prefix[];
 
-    const uint32_t expert = blockIdx.y;
-    uint32_t rows = p.M;
-    if (p.masked_m != nullptr) {
-        const int mm = __ldg(p.masked_m + expert);
-        rows = static_cast<uint32_t>(min(max(mm, 0), static_cast<int>(p.M)));
-    }
-    const uint32_t total = rows * p.segs;       // strips of this expert
-    const uint8_t *in = p.in + expert * p.in_expert_bytes;
-    uint8_t *out = p.out + expert * p.out_expert_bytes;
-    uint8_t *sc = p.scales + expert * p.scale_expert_bytes;
-
+    wait_for_producer();                        // before the first global access
     const uint32_t lane = threadIdx.x & 31u;
     const uint32_t warp = threadIdx.x >> 5;
-    const uint32_t sub = lane % L;              // lane within its group
+    ExpertTable t;
+    if constexpr (MULTI) {
+        t = make_table(p, smem_prefix, lane);
+    } else {
+        t.total = expert_strips(p, 0);
+    }
 
-    // Each warp owns an equal contiguous share [begin, end) of this expert's
-    // strips, so a one-wave grid finishes together (no partial last wave).
-    const uint64_t nwarps = static_cast<uint64_t>(gridDim.x) * kWarps;
-    const uint64_t wid = static_cast<uint64_t>(blockIdx.x) * kWarps + warp;
-    const uint32_t begin = static_cast<uint32_t>(wid * total / nwarps);
-    const uint32_t end = static_cast<uint32_t>((wid + 1) * total / nwarps);
-
-    uint32_t r0 = begin / p.segs;               // row and strip-in-row of s0
-    uint32_t sg0 = begin - r0 * p.segs;
-    for (uint32_t s0 = begin; s0 < end; s0 += ITEMS) {
-        uint32_t xr[ITEMS][8];
-        uint32_t ur[ITEMS][FUSED ? 8 : 1];
-        uint32_t row[ITEMS], col[ITEMS];
-        bool ok[ITEMS];
-
-        // -- issue every load of this iteration first ------------------------
-#pragma unroll
-        for (int k = 0; k < ITEMS; ++k) {
-            row[k] = r0;
-            col[k] = sg0 * kStripElems + lane * 16u;
-            ok[k] = (s0 + k < end) && (col[k] < p.K);
-            if (++sg0 == p.segs) {              // warp-uniform carry into the next row
-                sg0 = 0;
-                ++r0;
-            }
-            if (ok[k]) {
-                const uint8_t *src = in + static_cast<uint64_t>(row[k]) * p.in_row_bytes +
-                                     static_cast<uint64_t>(col[k]) * 2u;
-                load32B(src, xr[k]);
-                if constexpr (FUSED) load32B(src + static_cast<uint64_t>(p.K) * 2u, ur[k]);
-            } else {
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    xr[k][i] = 0u;
-                    if constexpr (FUSED) ur[k][i] = 0u;
-                }
-            }
-        }
-
-        // -- then the arithmetic, strip by strip ------------------------------
-#pragma unroll
-        for (int k = 0; k < ITEMS; ++k) {
-            if (s0 + k >= end) break;           // warp-uniform
-            float v[16];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                widen2<In>(xr[k][i], v[2 * i], v[2 * i + 1]);
-                if constexpr (FUSED) {
-                    float u0, u1;
-                    widen2<In>(ur[k][i], u0, u1);
-                    v[2 * i] = silu_mul(v[2 * i], u0);
-                    v[2 * i + 1] = silu_mul(v[2 * i + 1], u1);
-                }
-            }
-            float amax = 0.0f;
-#pragma unroll
-            for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
-#pragma unroll
-            for (int o = 1; o < L; o <<= 1)
-                amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
-
-            const GroupScale gs = make_scale<KIND>(amax);
-            uint32_t w[4];
-            encode16<KIND>(v, gs, w);
-
-            // group index within the row; every lane of a group agrees on it
-            const uint32_t g = col[k] / G;
-            uint32_t packed_word = 0;
-            if constexpr (KIND == Kind::E4M3_UE8M0) {
-                // assemble the little-endian word of groups 4j..4j+3 across the
-                // 4 groups' lanes (invalid groups contribute 0)
-                packed_word = ok[k] ? (gs.e8 << (8u * (g & 3u))) : 0u;
-                packed_word |= __shfl_xor_sync(0xFFFFFFFFu, packed_word, L);
-                packed_word |= __shfl_xor_sync(0xFFFFFFFFu, packed_word, 2 * L);
-            }
-            if (!ok[k]) continue;
-
-            store16B(out + static_cast<uint64_t>(row[k]) * p.K + col[k], w[0], w[1], w[2], w[3]);
-
-            if (sub == 0) {
-                const uint32_t r = row[k];
-                if (p.layout == kPacked) {
-                    if ((g & 3u) == 0u) {
-                        uint32_t *W = reinterpret_cast<uint32_t *>(sc);
-                        W[static_cast<uint64_t>(g >> 2) * p.mpad + r] = packed_word;
-                    }
-                } else {
-                    const uint64_t idx = (p.layout == kRowMajor)
-                                             ? static_cast<uint64_t>(r) * p.ng + g
-                                             : static_cast<uint64_t>(g) * p.mpad + r;
-                    if constexpr (KIND == Kind::E4M3_UE8M0)
-                        sc[idx] = static_cast<uint8_t>(gs.e8);
-                    else
-                        reinterpret_cast<float *>(sc)[idx] = gs.s;
-                }
-            }
-        }
+    // Block-cyclic schedule: a block is WARPS x items consecutive strips, CTA
+    // c takes blocks c, c + gridDim.x, ...; warp w takes the w-th `items`
+    // strips of each block.  All CTAs sweep the address space together, which
+    // keeps concurrent DRAM accesses close (row-buffer locality).
+    const uint32_t items = p.items;             // 1 .. ITEMS (launch-time)
+    const uint32_t block = WARPS * items;
+    const uint32_t nblocks = (t.total + block - 1) / block;
+    for (uint32_t blk = blockIdx.x; blk < nblocks; blk += gridDim.x) {
+        const uint32_t s = blk * block + warp * items;
+        if (s >= t.total) break;                // warp-uniform
+        Chunk<ITEMS, FUSED> ch;
+        load_chunk<ITEMS, FUSED, MULTI>(ch, s, min(items, t.total - s), t, p, lane);
+        quantize_chunk<In, G, KIND, FUSED, ITEMS>(ch, p, lane);
     }
     release_dependents();
 }

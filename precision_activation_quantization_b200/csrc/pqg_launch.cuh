@@ -1,6 +1,7 @@
 // Host-side launch of the quantization kernel family: picks the compile-time
-// variant, sizes the grid and launches with cudaLaunchKernelEx on the caller's
-// stream (with the programmatic-dependent-launch attribute when enabled).
+// variant, sizes the grid and the dynamic shared memory, and launches with
+// cudaLaunchKernelEx on the caller's stream (with the programmatic-dependent-
+// launch attribute when enabled).
 #pragma once
 
 #include <cuda_runtime.h>
@@ -9,15 +10,16 @@
 #include <cstdint>
 
 #include "pqg_kernel.cuh"
+#include "pqg_row_kernel.cuh"
 
 namespace pqg {
 
 // Everything the launcher needs, already validated by the C-ABI shim.
 struct LaunchArgs {
     Params p;
-    uint32_t experts;       // grid.y
-    uint32_t grid_rows;     // rows per expert the grid is sized for
-    int group;              // 32 / 64 / 128
+    uint64_t expected_strips;  // strips the grid is sized for (all experts)
+    uint64_t expected_rows;    // rows the grid is sized for (per-token kernel)
+    int group;                 // 32 / 64 / 128, or K (per-token)
     Kind kind;
     bool fused;
     bool pdl;
@@ -26,29 +28,50 @@ struct LaunchArgs {
 
 int sm_count(int device);  // cached cudaDevAttrMultiProcessorCount
 
-// Strips each warp takes per iteration: each lane keeps this many 32-byte
-// loads in flight (twice as many when fused).  Tunable at build time.
+// Strips per register chunk (ITEMS) and warps per CTA, tunable at build time.
+// Each lane issues ITEMS 32-byte loads (twice that fused) per chunk.
 #ifndef PQG_ITEMS_PLAIN
 #define PQG_ITEMS_PLAIN 2
 #endif
-#ifndef PQG_ITEMS_FUSED
-#define PQG_ITEMS_FUSED 2
+#ifndef PQG_WARPS_PLAIN
+#define PQG_WARPS_PLAIN 8
 #endif
+#ifndef PQG_ITEMS_FUSED
+#define PQG_ITEMS_FUSED 1
+#endif
+#ifndef PQG_WARPS_FUSED
+#define PQG_WARPS_FUSED 8
+#endif
+
+// Grid cap in waves of resident CTAs, and the size (in waves of blocks) up to
+// which a call runs as a single looping wave.
+#ifndef PQG_WAVES
+#define PQG_WAVES 8
+#endif
+#ifndef PQG_SHORT_WAVES
+#define PQG_SHORT_WAVES 4
+#endif
+
 template <bool FUSED>
-constexpr int items_per_warp() {
-    return FUSED ? PQG_ITEMS_FUSED : PQG_ITEMS_PLAIN;
-}
+struct Shape {
+    static constexpr int kItems = FUSED ? PQG_ITEMS_FUSED : PQG_ITEMS_PLAIN;
+    static constexpr int kWarps = FUSED ? PQG_WARPS_FUSED : PQG_WARPS_PLAIN;
+};
 
-template <typename In, int G, Kind KIND, bool FUSED>
+template <typename In, int G, Kind KIND, bool FUSED, bool MULTI>
 cudaError_t launch_variant(const LaunchArgs &a) {
-    constexpr int ITEMS = items_per_warp<FUSED>();
-    auto kernel = quant_kernel<In, G, KIND, FUSED, ITEMS>;
+    using Sh = Shape<FUSED>;
+    constexpr int kThreads = Sh::kWarps * 32;
+    auto kernel = quant_kernel<In, G, KIND, FUSED, Sh::kItems, Sh::kWarps, MULTI>;
 
-    // resident CTAs per SM for this variant (queried once per variant)
+    // Resident CTAs per SM, queried once per variant for the largest expert
+    // table (16 KB of shared memory); registers are the binding limit.
     static const int blocks_per_sm = [&] {
         int n = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, kThreads, 0) !=
-                cudaSuccess ||
+        if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(smem_bytes(kMaxExperts))) != cudaSuccess ||
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, kThreads,
+                                                          smem_bytes(kMaxExperts)) != cudaSuccess ||
             n < 1)
             n = 1;
         return n;
@@ -58,41 +81,133 @@ cudaError_t launch_variant(const LaunchArgs &a) {
     cudaError_t err = cudaGetDevice(&device);
     if (err != cudaSuccess) return err;
 
-    // One wave of resident CTAs at most; fewer when the work is small, so that
-    // every warp has at least ITEMS strips.
-    const uint64_t strips = static_cast<uint64_t>(a.grid_rows) * a.p.segs;
-    const uint64_t per_cta = static_cast<uint64_t>(kWarps) * ITEMS;
-    uint64_t ctas = (strips + per_cta - 1) / per_cta;
-    uint64_t wave = static_cast<uint64_t>(sm_count(device)) * blocks_per_sm;
-    if (a.experts > 1) wave = (wave + a.experts - 1) / a.experts;
-    if (ctas > wave) ctas = wave;
+    // Strips per warp: ITEMS, or 1 when the expected work would not fill one
+    // wave (latency-bound calls spread over more SMs).  Grid: one CTA per
+    // block of the expected work, but a short call (at most PQG_SHORT_WAVES
+    // waves of blocks) runs one resident wave that loops over the blocks (no
+    // ragged last wave), and a long one at most PQG_WAVES waves.  Blocks are
+    // taken round-robin, so any real total is covered.
+    const uint64_t wave = static_cast<uint64_t>(sm_count(device)) * blocks_per_sm;
+    Params p = a.p;
+    p.items = Sh::kItems;
+    if (a.expected_strips < wave * Sh::kWarps * Sh::kItems) p.items = 1;
+    const uint64_t per_cta = static_cast<uint64_t>(Sh::kWarps) * p.items;
+    uint64_t ctas = (a.expected_strips + per_cta - 1) / per_cta;
+    const uint64_t cap = ctas <= wave * PQG_SHORT_WAVES ? wave : wave * PQG_WAVES;
+    if (ctas > cap) ctas = cap;
     if (ctas < 1) ctas = 1;
 
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(ctas), a.experts, 1);
+    cfg.gridDim = dim3(static_cast<unsigned>(ctas), 1, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
-    cfg.dynamicSmemBytes = 0;
+    cfg.dynamicSmemBytes = smem_bytes(a.p.experts);
     cfg.stream = a.stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = a.pdl ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, kernel, a.p);
+    return cudaLaunchKernelEx(&cfg, kernel, p);
+}
+
+template <typename In, int G, Kind KIND>
+cudaError_t launch_kind(const LaunchArgs &a) {
+    const bool multi = a.p.experts > 1;
+    if (a.fused)
+        return multi ? launch_variant<In, G, KIND, true, true>(a)
+                     : launch_variant<In, G, KIND, true, false>(a);
+    return multi ? launch_variant<In, G, KIND, false, true>(a)
+                 : launch_variant<In, G, KIND, false, false>(a);
 }
 
 template <typename In, int G>
 cudaError_t launch_group(const LaunchArgs &a) {
     switch (a.kind) {
+        case Kind::E4M3_FP32: return launch_kind<In, G, Kind::E4M3_FP32>(a);
+        case Kind::E4M3_UE8M0: return launch_kind<In, G, Kind::E4M3_UE8M0>(a);
+        case Kind::INT8_FP32: return launch_kind<In, G, Kind::INT8_FP32>(a);
+    }
+    return cudaErrorInvalidValue;
+}
+
+// ---------------------------------------------------------------------------
+// Per-token (G = K) launches
+// ---------------------------------------------------------------------------
+
+// Warps sharing a row and 16-element slots per thread for a row of K outputs.
+inline void row_shape(uint32_t K, uint32_t *wpr, int *slots) {
+    const uint32_t nslots = K / 16u;
+    if (nslots <= 32) { *wpr = 1; *slots = 1; }
+    else if (nslots <= 64) { *wpr = 1; *slots = 2; }
+    else if (nslots <= 128) { *wpr = 1; *slots = 4; }
+    else if (nslots <= 256) { *wpr = 2; *slots = 4; }
+    else if (nslots <= 512) { *wpr = 4; *slots = 4; }
+    else { *wpr = 8; *slots = 4; }
+}
+
+template <typename In, Kind KIND, bool FUSED, int SLOTS>
+cudaError_t launch_row_variant(const LaunchArgs &a, uint32_t wpr) {
+    auto kernel = row_quant_kernel<In, KIND, FUSED, SLOTS>;
+    static const int blocks_per_sm = [&] {
+        int n = 0;
+        if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(smem_bytes(kMaxExperts))) != cudaSuccess ||
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, kRowThreads,
+                                                          smem_bytes(kMaxExperts)) != cudaSuccess ||
+            n < 1)
+            n = 1;
+        return n;
+    }();
+    int device = 0;
+    cudaError_t err = cudaGetDevice(&device);
+    if (err != cudaSuccess) return err;
+
+    Params p = a.p;
+    p.segs = 1;        // the expert table counts rows
+    p.items = wpr;     // warps per row
+    const uint64_t rows_per_cta = (kRowThreads / 32) / wpr;
+    uint64_t ctas = (a.expected_rows + rows_per_cta - 1) / rows_per_cta;
+    const uint64_t cap = static_cast<uint64_t>(sm_count(device)) * blocks_per_sm * PQG_WAVES;
+    if (ctas > cap) ctas = cap;
+    if (ctas < 1) ctas = 1;
+
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(ctas), 1, 1);
+    cfg.blockDim = dim3(kRowThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem_bytes(a.p.experts);
+    cfg.stream = a.stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = a.pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kernel, p);
+}
+
+template <typename In, Kind KIND, bool FUSED>
+cudaError_t launch_row_kind(const LaunchArgs &a) {
+    uint32_t wpr = 1;
+    int slots = 1;
+    row_shape(a.p.K, &wpr, &slots);
+    switch (slots) {
+        case 1: return launch_row_variant<In, KIND, FUSED, 1>(a, wpr);
+        case 2: return launch_row_variant<In, KIND, FUSED, 2>(a, wpr);
+        default: return launch_row_variant<In, KIND, FUSED, 4>(a, wpr);
+    }
+}
+
+template <typename In>
+cudaError_t launch_row(const LaunchArgs &a) {
+    switch (a.kind) {
         case Kind::E4M3_FP32:
-            return a.fused ? launch_variant<In, G, Kind::E4M3_FP32, true>(a)
-                           : launch_variant<In, G, Kind::E4M3_FP32, false>(a);
+            return a.fused ? launch_row_kind<In, Kind::E4M3_FP32, true>(a)
+                           : launch_row_kind<In, Kind::E4M3_FP32, false>(a);
         case Kind::E4M3_UE8M0:
-            return a.fused ? launch_variant<In, G, Kind::E4M3_UE8M0, true>(a)
-                           : launch_variant<In, G, Kind::E4M3_UE8M0, false>(a);
+            return a.fused ? launch_row_kind<In, Kind::E4M3_UE8M0, true>(a)
+                           : launch_row_kind<In, Kind::E4M3_UE8M0, false>(a);
         case Kind::INT8_FP32:
-            return a.fused ? launch_variant<In, G, Kind::INT8_FP32, true>(a)
-                           : launch_variant<In, G, Kind::INT8_FP32, false>(a);
+            return a.fused ? launch_row_kind<In, Kind::INT8_FP32, true>(a)
+                           : launch_row_kind<In, Kind::INT8_FP32, false>(a);
     }
     return cudaErrorInvalidValue;
 }
@@ -104,7 +219,7 @@ cudaError_t launch_dtype(const LaunchArgs &a) {
         case 64: return launch_group<In, 64>(a);
         case 128: return launch_group<In, 128>(a);
     }
-    return cudaErrorInvalidValue;
+    return launch_row<In>(a);   // per-token: group == K (checked by the caller)
 }
 
 cudaError_t launch_bf16(const LaunchArgs &a);

@@ -1,0 +1,128 @@
+// Per-token quantization (one group per row, G = K) for sm_100a.
+//
+// The TeleFuser "tf-kernel 安装与使用" page (使用示例) shows the per-token form
+// of the operation, tf_per_token_quant_fp8(x, x_q, x_scale): one fp32 scale per
+// row ([M, 1]) and E4M3 codes into caller-allocated outputs.  The arithmetic is
+// the per-group rule with the group widened to the whole row.
+//
+// A row is shared by WPR warps (1, 2, 4 or 8, chosen at launch so that a
+// thread holds at most SLOTS 16-element slots).  Lanes read consecutive
+// 32-byte slots, so a warp's loads cover 1 KB contiguous.  The row absmax is a
+// warp xor-reduction, then (WPR > 1) one exchange through shared memory.  The
+// partials are double-buffered by iteration parity, so one __syncthreads per
+// row iteration is enough.  Values stay in registers between the reduction and
+// the quantization, so every input byte is read once.  Rows come from the same
+// expert table as the strip kernel (counting rows instead of strips), so flat,
+// batched and masked dispatch and the fused SiLU-and-mul all work unchanged.
+#pragma once
+
+#include "pqg_kernel.cuh"
+
+namespace pqg {
+
+constexpr int kRowThreads = 256;  // 8 warps per CTA
+
+template <typename In, Kind KIND, bool FUSED, int SLOTS>
+__global__ void __launch_bounds__(kRowThreads)
+    row_quant_kernel(const __grid_constant__ Params p) {
+    extern __shared__ __align__(16) uint32_t smem_prefix[];
+    __shared__ float partial[2][kRowThreads / 32];
+
+    wait_for_producer();                        // before the first global access
+    const uint32_t lane = threadIdx.x & 31u;
+    const uint32_t warp = threadIdx.x >> 5;
+    // p.segs is 1 for this kernel: the table counts rows
+    const ExpertTable t = make_table(p, smem_prefix, lane);
+
+    const uint32_t wpr = p.items;               // warps per row: 1, 2, 4 or 8
+    const uint32_t rows_per_iter = (kRowThreads / 32) / wpr;
+    const uint32_t sub = warp / wpr;            // this warp's row within the iteration
+    const uint32_t wr = warp - sub * wpr;       // warp index within the row
+    const uint32_t tpr = wpr * 32u;             // threads per row
+    const uint32_t tid = wr * 32u + lane;       // thread index within the row
+    const uint32_t nslots = p.K / 16u;          // 16-element slots per row
+
+    uint32_t parity = 0;
+    for (uint32_t base = blockIdx.x * rows_per_iter; base < t.total;
+         base += gridDim.x * rows_per_iter, parity ^= 1u) {
+        const uint32_t r = base + sub;          // warp-uniform
+        const bool live = r < t.total;
+        Span sp = locate(t, p.experts, live ? r : 0u);
+        const uint32_t row = (live ? r : 0u) - sp.start;
+        const uint8_t *src = p.in + sp.e * p.in_expert_bytes +
+                             static_cast<uint64_t>(row) * p.in_row_bytes;
+
+        // -- loads, then widen (and fuse) into registers -----------------------
+        uint32_t x[SLOTS][8];
+        uint32_t u[SLOTS][FUSED ? 8 : 1];
+#pragma unroll
+        for (int j = 0; j < SLOTS; ++j) {
+            const uint32_t slot = tid + j * tpr;
+            if (live && slot < nslots) {
+                load32B(src + slot * 32u, x[j]);
+                if constexpr (FUSED) load32B(src + static_cast<uint64_t>(p.K) * 2u + slot * 32u, u[j]);
+            } else {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    x[j][i] = 0u;
+                    if constexpr (FUSED) u[j][i] = 0u;
+                }
+            }
+        }
+        float v[SLOTS][16];
+        float amax = 0.0f;
+#pragma unroll
+        for (int j = 0; j < SLOTS; ++j) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                widen2<In>(x[j][i], v[j][2 * i], v[j][2 * i + 1]);
+                if constexpr (FUSED) {
+                    float u0, u1;
+                    widen2<In>(u[j][i], u0, u1);
+                    v[j][2 * i] = silu_mul(v[j][2 * i], u0);
+                    v[j][2 * i + 1] = silu_mul(v[j][2 * i + 1], u1);
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[j][i]));
+        }
+
+        // -- row absmax: warp, then across the row's warps ---------------------
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+        if (wpr > 1) {
+            if (lane == 0) partial[parity][warp] = amax;
+            __syncthreads();
+            for (uint32_t w = 0; w < wpr; ++w) amax = fmaxf(amax, partial[parity][sub * wpr + w]);
+        }
+
+        // -- scale, codes, stores ----------------------------------------------
+        const GroupScale gs = make_scale<KIND>(amax);
+        if (live) {
+            uint8_t *dst = p.out + sp.e * p.out_expert_bytes + static_cast<uint64_t>(row) * p.K;
+#pragma unroll
+            for (int j = 0; j < SLOTS; ++j) {
+                const uint32_t slot = tid + j * tpr;
+                if (slot < nslots) {
+                    uint32_t w[4];
+                    encode16<KIND>(v[j], gs, w);
+                    store16B(dst + slot * 16u, w[0], w[1], w[2], w[3]);
+                }
+            }
+            if (tid == 0) {
+                // one group per row: row-major, column-major and packed all put
+                // row r's scale at element / word r of the expert's plane
+                uint8_t *sc = p.scales + sp.e * p.scale_expert_bytes;
+                if (p.layout == kPacked)
+                    reinterpret_cast<uint32_t *>(sc)[row] = gs.e8;  // bytes 1..3 are 0
+                else if constexpr (KIND == Kind::E4M3_UE8M0)
+                    sc[row] = static_cast<uint8_t>(gs.e8);
+                else
+                    reinterpret_cast<float *>(sc)[row] = gs.s;
+            }
+        }
+    }
+    release_dependents();
+}
+
+}  // namespace pqg

@@ -110,6 +110,12 @@ def test_scales_bytes_matches_oracle(E, M, K, G, fmt, layout):
     assert int(np.prod(shape)) * torch.empty((), dtype=dt).element_size() == want
 
 
+def test_per_token_scales_bytes():
+    for K in (80, 7168, 16384):
+        assert pqg.pqg_scales_bytes(1, 5, K, K, pqg.PQG_SCALE_FP32, pqg.PQG_ROW_MAJOR) == 5 * 4
+        assert pqg.pqg_scales_bytes(2, 5, K, K, pqg.PQG_SCALE_UE8M0, pqg.PQG_UE8M0_PACKED) == 2 * 8 * 4
+
+
 def test_scales_bytes_rejects():
     S, R, C, P = pqg.PQG_SCALE_FP32, pqg.PQG_ROW_MAJOR, pqg.PQG_COL_MAJOR_TMA, pqg.PQG_UE8M0_PACKED
     assert pqg.pqg_scales_bytes(1, 4, 256, 128, S, P) == pqg.PQG_ERR_UNSUPPORTED
@@ -144,12 +150,17 @@ def call(**kw):
     (dict(scale_layout=-1), pqg.PQG_ERR_INVALID_ARG),
     (dict(group=0), pqg.PQG_ERR_INVALID_ARG),
     (dict(group=16), pqg.PQG_ERR_UNSUPPORTED),
-    (dict(group=256), pqg.PQG_ERR_UNSUPPORTED),
+    (dict(group=256, K=512), pqg.PQG_ERR_UNSUPPORTED),
+    (dict(group=512, K=1024), pqg.PQG_ERR_UNSUPPORTED),          # neither 32/64/128 nor K
+    (dict(group=16400, K=16400), pqg.PQG_ERR_UNSUPPORTED),       # per-token K > 16384
+    (dict(group=200, K=200), pqg.PQG_ERR_UNSUPPORTED),           # per-token K % 16 != 0
     (dict(K=200), pqg.PQG_ERR_INVALID_ARG),
     (dict(K=-256), pqg.PQG_ERR_INVALID_ARG),
     (dict(M=-1), pqg.PQG_ERR_INVALID_ARG),
     (dict(num_experts=0), pqg.PQG_ERR_INVALID_ARG),
     (dict(num_experts=70000), pqg.PQG_ERR_INVALID_ARG),
+    (dict(num_experts=4097), pqg.PQG_ERR_INVALID_ARG),
+    (dict(num_experts=4096, M=1 << 12, K=1 << 14), pqg.PQG_ERR_INVALID_ARG),  # 2^31 strips
     (dict(out_dtype=pqg.PQG_INT8, scale_fmt=pqg.PQG_SCALE_UE8M0), pqg.PQG_ERR_UNSUPPORTED),
     (dict(scale_layout=pqg.PQG_UE8M0_PACKED), pqg.PQG_ERR_UNSUPPORTED),
     (dict(in_ptr=0), pqg.PQG_ERR_INVALID_ARG),

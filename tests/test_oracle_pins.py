@@ -321,7 +321,8 @@ def test_int8_dequant_error_bound():
     assert q.view(np.int8).max() == 127 or q.view(np.int8).min() == -127
 
 
-@pytest.mark.parametrize("in_dtype,group", [("bf16", 128), ("fp16", 64), ("bf16", 32)])
+@pytest.mark.parametrize("in_dtype,group", [("bf16", 128), ("fp16", 64), ("bf16", 32),
+                                            ("bf16", 1024), ("fp16", 1024)])
 def test_whole_path_matches_torch_composition(in_dtype, group):
     """fp32-scale E4M3 path against torch primitives (amax, fp32 division, fp8 cast)."""
     w = inputs.sweep(M=64, K=1024, in_dtype=in_dtype, group=group)

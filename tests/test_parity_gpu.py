@@ -23,13 +23,13 @@ KINDS = [  # (out_dtype, scale_fmt, layout)
 
 
 def hard_input(shape, seed, in_dtype="bf16"):
-    """N(0,1) rows with per-row magnitudes over many binades, all-zero groups of
-    32, -0.0 entries, outliers and subnormal inputs."""
+    """N(0,1) rows with per-row magnitudes over many binades, all-zero runs of
+    16, -0.0 entries, outliers and subnormal inputs."""
     rng = np.random.default_rng(seed)
     x = rng.standard_normal(shape).astype(np.float32)
     lo, hi = (-20, 10) if in_dtype == "bf16" else (-12, 6)
     x *= np.exp2(rng.uniform(lo, hi, shape[:-1] + (1,))).astype(np.float32)
-    flat = x.reshape(-1, 32)
+    flat = x.reshape(-1, 16)
     flat[rng.random(flat.shape[0]) < 1 / 16] = 0.0
     x[rng.random(shape) < 0.01] = -0.0
     out = rng.random(shape) < 0.005
@@ -239,3 +239,68 @@ def test_torch_helper_matches_raw_call():
     assert_same(s.view(torch.uint8).cpu().numpy().reshape(-1), rs, "scales")
     with pytest.raises(pqg.PqgError):
         pqg.quant(x, group=128, out_dtype="int8", scale_fmt="ue8m0")
+
+
+# --------------------------------------------------------------------------
+# the balanced scheduler and its expert table
+# --------------------------------------------------------------------------
+
+def test_masked_skewed_counts():
+    """One full expert among many empty or tiny ones: every strip lands once."""
+    E, M, K = 40, 96, 1536
+    mm = np.zeros(E, np.int32)
+    mm[7], mm[8], mm[39], mm[20] = M, 1, 3, 95
+    for fused in (False, True):
+        w = make(M, K, 128, ("e4m3", "ue8m0", "packed"), fused=fused, E=E, seed=21,
+                 masked_m=mm, expected_m=2)
+        if fused:
+            check_fused(w, max_flip_frac=1e-3)
+        else:
+            check_exact(w)
+
+
+def test_masked_many_experts():
+    """The largest expert table (4096 entries) with 0/1/2 rows each."""
+    E, M, K = 4096, 2, 128
+    mm = np.random.default_rng(22).integers(0, 3, size=E).astype(np.int32)
+    check_exact(make(M, K, 64, ("int8", "fp32", "col"), E=E, seed=23, masked_m=mm, expected_m=1))
+
+
+@pytest.mark.parametrize("E", [2, 31, 32, 33, 64])
+def test_expert_table_modes(E):
+    """Warp-register table (E <= 32) and shared-memory table (E > 32) agree
+    with the oracle, including empty experts next to full ones."""
+    M, K = 24, 1024
+    mm = np.random.default_rng(30 + E).integers(-2, M + 3, size=E).astype(np.int32)
+    mm[0], mm[-1] = 0, M
+    check_exact(make(M, K, 64, ("e4m3", "ue8m0", "packed"), E=E, seed=31, masked_m=mm,
+                     expected_m=3))
+    check_fused(make(M, K, 128, ("e4m3", "fp32", "col"), fused=True, E=E, seed=32, masked_m=mm,
+                     expected_m=M), max_flip_frac=1e-3)
+
+
+# --------------------------------------------------------------------------
+# per-token quantization (one group per row, G = K)
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("K", [80, 512, 1024, 2048, 4096, 7168, 16384])
+@pytest.mark.parametrize("kind", KINDS, ids=lambda k: "_".join(k))
+def test_per_token_bit_exact(K, kind):
+    for M, in_dtype in [(37, "bf16"), (5, "fp16")]:
+        check_exact(make(M, K, K, kind, in_dtype, seed=K + M))
+
+
+@pytest.mark.parametrize("K", [256, 2048, 7168])
+def test_per_token_fused_and_masked(K):
+    E, M = 5, 19
+    mm = np.array([0, 19, 1, 40, 7], np.int32)
+    check_fused(make(M, K, K, ("e4m3", "fp32", "row"), fused=True, seed=K, E=E, masked_m=mm,
+                     expected_m=4), max_flip_frac=1e-3)
+    check_exact(make(M, K, K, ("e4m3", "ue8m0", "packed"), seed=K + 1, E=E, masked_m=mm,
+                     expected_m=4))
+    check_exact(make(300, K, K, ("int8", "fp32", "col"), in_dtype="fp16", seed=K + 2))
+
+
+def test_per_token_full_size():
+    w = inputs.flat_hidden(layout="row", scale_fmt="fp32").with_(group=7168)
+    check_exact(w)

@@ -100,12 +100,23 @@ enum pqg_scale_fmt {
  *                       group 4j + b; bytes for groups >= ng are written 0.
  *                       UE8M0 only ("aligned" in the pages' trait list means
  *                       ng % 4 == 0, i.e. no partial last word).
+ *   PQG_UE8M0_TILED_128x4 : the 128x4 block-scale tile ("F8_128x4", the 1D
+ *                       swizzled layout the FlashInfer notes name for mm_mxfp8,
+ *                       section 6).  Rows in tiles of 128, groups in tiles of 4;
+ *                       one 512-byte tile per (row tile, group tile), tiles in
+ *                       row-tile-major order; inside a tile the exponent of
+ *                       (row m, group g) is byte (m%32)*16 + ((m/32)%4)*4 + g%4.
+ *                       Plane: ceil(M/128)*128 x ceil(ng/4)*4 bytes.  Bytes of
+ *                       padding groups (>= ng) in a quantized row are written 0;
+ *                       padding rows are not written.  UE8M0 only; with G = 32
+ *                       this is the MXFP8 operand format.
  * Expert e's plane starts pqg_scales_bytes(1, M, K, ...) * e bytes into the
  * buffer. */
 enum pqg_scale_layout {
     PQG_ROW_MAJOR = 0,
     PQG_COL_MAJOR_TMA = 1,
-    PQG_UE8M0_PACKED = 2
+    PQG_UE8M0_PACKED = 2,
+    PQG_UE8M0_TILED_128x4 = 3
 };
 
 /*
@@ -129,7 +140,8 @@ enum pqg_scale_layout {
  *          K a multiple of 16, at most 16384).
  * in_dtype PQG_BF16 or PQG_FP16.   out_dtype PQG_E4M3 or PQG_INT8.
  * scale_fmt, scale_layout   see above.  PQG_SCALE_UE8M0 requires PQG_E4M3, and
- *          PQG_UE8M0_PACKED requires PQG_SCALE_UE8M0 (else PQG_ERR_UNSUPPORTED).
+ *          PQG_UE8M0_PACKED and PQG_UE8M0_TILED_128x4 require PQG_SCALE_UE8M0
+ *          (else PQG_ERR_UNSUPPORTED).
  * fuse_silu_mul  nonzero: quantize silu(gate) * up (see the numerics above).
  * masked_m device, int32[num_experts], or NULL.  Masked dispatch (grouped-masked
  *          MoE): expert e quantizes only rows m < clamp(masked_m[e], 0, M); the

@@ -30,7 +30,7 @@ _LIB_PATH = os.path.join(_HERE, "liboracle.so")
 _LOCK = threading.Lock()
 _lib = None
 
-LAYOUTS = {"row": 0, "col": 1, "packed": 2}
+LAYOUTS = {"row": 0, "col": 1, "packed": 2, "tile128x4": 3}
 
 
 def build(force: bool = False, src: str = _SRC, out: str = _LIB_PATH) -> str:
@@ -176,6 +176,8 @@ def scales_shape(E: int, M: int, K: int, group: int, scale_fmt: str, layout: str
         shape = (E, M, ng)
     elif layout == "col":
         shape = (E, ng, mpad)
+    elif layout == "tile128x4":
+        return (E, (M + 127) // 128 * ((ng + 3) // 4) * 512), np.uint8
     else:
         return (E, (ng + 3) // 4, mpad), np.int32
     return shape, (np.uint8 if scale_fmt == "ue8m0" else np.float32)

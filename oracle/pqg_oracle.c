@@ -41,6 +41,13 @@
  *   - the UE8M0-packed layout stores the exponents of groups 4j..4j+3 of a
  *     row in one little-endian int32 word; bytes for groups past the last one
  *     are 0.
+ *   - the 128x4 tiled layout ("F8_128x4", the 1D swizzled block-scale layout
+ *     the FlashInfer notes name for mm_mxfp8, section 6) is read as the public
+ *     block-scale tile: rows in tiles of 128, scale columns in tiles of 4, one
+ *     512-byte tile per (row tile, column tile) in row-tile-major order, and
+ *     inside a tile the exponent of (row m, group g) at byte
+ *     (m % 32) * 16 + ((m / 32) % 4) * 4 + (g % 4).  Bytes of padding columns
+ *     (groups >= ng) in a quantized row are 0; padding rows are not written.
  *
  * Build: gcc -O2 -std=c11 -fPIC -shared -ffp-contract=off (no fast-math).
  * Floating point: C float arithmetic is IEEE binary32 with round-to-nearest
@@ -58,7 +65,7 @@
 #define PQGO_EPS 1e-10f         /* absmax floor ([PR] "不低于 EPS")             */
 
 /* layouts understood by the oracle (numbered for the Python wrapper) */
-enum { PQGO_ROW = 0, PQGO_COL = 1, PQGO_PACKED = 2 };
+enum { PQGO_ROW = 0, PQGO_COL = 1, PQGO_PACKED = 2, PQGO_TILE128X4 = 3 };
 
 /* ------------------------------------------------------------------------ */
 /* Input decoding                                                            */
@@ -183,6 +190,14 @@ int8_t pqgo_int8_encode(float t) {
 /* rows of one expert's column-major scale plane: M rounded up to 4 */
 static int64_t padded_rows(int64_t M) { return (M + 3) / 4 * 4; }
 
+/* byte offset of (row m, group g) in one expert's 128x4-tiled plane */
+static int64_t tile128x4_offset(int64_t m, int64_t g, int64_t ng) {
+    int64_t col_tiles = (ng + 3) / 4;
+    int64_t tile = (m / 128) * col_tiles + (g / 4);
+    int64_t r = m % 128;
+    return tile * 512 + (r % 32) * 16 + (r / 32) * 4 + (g % 4);
+}
+
 /* Size in bytes of the scale buffer for E experts of M rows of K outputs. */
 int64_t pqgo_scales_nbytes(int64_t E, int64_t M, int64_t K, int G,
                            int scale_ue8m0, int layout) {
@@ -190,6 +205,7 @@ int64_t pqgo_scales_nbytes(int64_t E, int64_t M, int64_t K, int G,
     int64_t elem = scale_ue8m0 ? 1 : 4;
     if (layout == PQGO_ROW) return E * M * ng * elem;
     if (layout == PQGO_COL) return E * ng * padded_rows(M) * elem;
+    if (layout == PQGO_TILE128X4) return E * ((M + 127) / 128) * ((ng + 3) / 4) * 512;
     /* packed: int32 words, ceil(ng / 4) per row */
     return E * ((ng + 3) / 4) * padded_rows(M) * 4;
 }
@@ -211,9 +227,9 @@ int pqgo_quant(const uint16_t *in, uint8_t *out, void *scales, int64_t E,
                int scale_ue8m0, int layout, int fused,
                const int32_t *masked_m) {
     if (E < 1 || M < 0 || K <= 0 || G <= 0 || K % G != 0) return -1;
-    if (layout < PQGO_ROW || layout > PQGO_PACKED) return -1;
+    if (layout < PQGO_ROW || layout > PQGO_TILE128X4) return -1;
     if (scale_ue8m0 && out_int8) return -1;       /* UE8M0 pairs with FMAX */
-    if (layout == PQGO_PACKED && !scale_ue8m0) return -1;
+    if ((layout == PQGO_PACKED || layout == PQGO_TILE128X4) && !scale_ue8m0) return -1;
 
     const int64_t ng = K / G;
     const int64_t in_width = fused ? 2 * K : K;
@@ -273,11 +289,20 @@ int pqgo_quant(const uint16_t *in, uint8_t *out, void *scales, int64_t E,
                     int64_t idx = e * ng * mpad + g * mpad + m;
                     if (scale_ue8m0) ((uint8_t *)scales)[idx] = (uint8_t)ebyte;
                     else ((float *)scales)[idx] = s;
-                } else {
+                } else if (layout == PQGO_PACKED) {
                     int64_t nwords = (ng + 3) / 4;
                     int64_t word = e * nwords * mpad + (g / 4) * mpad + m;
                     ((uint8_t *)scales)[word * 4 + (g % 4)] = (uint8_t)ebyte;
+                } else {
+                    int64_t plane = ((M + 127) / 128) * ((ng + 3) / 4) * 512;
+                    ((uint8_t *)scales)[e * plane + tile128x4_offset(m, g, ng)] = (uint8_t)ebyte;
                 }
+            }
+            /* 128x4 tiles: padding columns of this row are 0 */
+            if (status == 0 && layout == PQGO_TILE128X4 && ng % 4 != 0) {
+                int64_t plane = ((M + 127) / 128) * ((ng + 3) / 4) * 512;
+                for (int64_t g = ng; g < (ng + 3) / 4 * 4; ++g)
+                    ((uint8_t *)scales)[e * plane + tile128x4_offset(m, g, ng)] = 0;
             }
             /* packed words: exponent bytes of groups past the last are 0 */
             if (status == 0 && layout == PQGO_PACKED && ng % 4 != 0) {

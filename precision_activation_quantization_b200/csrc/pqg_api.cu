@@ -33,13 +33,14 @@ int check_geometry(int64_t num_experts, int64_t M, int64_t K, int group, int sca
                    int scale_layout, int64_t *plane) {
     if (scale_fmt != PQG_SCALE_FP32 && scale_fmt != PQG_SCALE_UE8M0) return PQG_ERR_INVALID_ARG;
     if (scale_layout != PQG_ROW_MAJOR && scale_layout != PQG_COL_MAJOR_TMA &&
-        scale_layout != PQG_UE8M0_PACKED)
+        scale_layout != PQG_UE8M0_PACKED && scale_layout != PQG_UE8M0_TILED_128x4)
         return PQG_ERR_INVALID_ARG;
     if (group <= 0) return PQG_ERR_INVALID_ARG;
     // G in {32, 64, 128}, or one group per row (per-token, K <= 16384)
     const bool per_token = group == K && K % 16 == 0 && K <= kMaxPerTokenK;
     if (group != 32 && group != 64 && group != 128 && !per_token) return PQG_ERR_UNSUPPORTED;
-    if (scale_layout == PQG_UE8M0_PACKED && scale_fmt != PQG_SCALE_UE8M0)
+    if ((scale_layout == PQG_UE8M0_PACKED || scale_layout == PQG_UE8M0_TILED_128x4) &&
+        scale_fmt != PQG_SCALE_UE8M0)
         return PQG_ERR_UNSUPPORTED;
     if (num_experts < 1 || num_experts > static_cast<int64_t>(pqg::kMaxExperts))
         return PQG_ERR_INVALID_ARG;
@@ -57,8 +58,10 @@ int check_geometry(int64_t num_experts, int64_t M, int64_t K, int group, int sca
         *plane = M * ng * elem;
     else if (scale_layout == PQG_COL_MAJOR_TMA)
         *plane = ng * padded_rows(M) * elem;
-    else
+    else if (scale_layout == PQG_UE8M0_PACKED)
         *plane = (ng + 3) / 4 * padded_rows(M) * 4;
+    else
+        *plane = (M + 127) / 128 * ((ng + 3) / 4) * 512;
     return PQG_OK;
 }
 

@@ -56,7 +56,23 @@ namespace pqg {
 enum class Kind : int { E4M3_FP32 = 0, E4M3_UE8M0 = 1, INT8_FP32 = 2 };
 
 // Runtime scale layouts (same numbering as the C ABI's pqg_scale_layout).
-enum : uint32_t { kRowMajor = 0, kColMajor = 1, kPacked = 2 };
+enum : uint32_t { kRowMajor = 0, kColMajor = 1, kPacked = 2, kTiled128x4 = 3 };
+
+// Byte of (row m, group g) in one expert's 128x4-tiled exponent plane.
+__device__ __forceinline__ uint64_t tile128x4_offset(uint32_t m, uint32_t g, uint32_t ng) {
+    const uint32_t col_tiles = (ng + 3u) >> 2;
+    const uint64_t tile = static_cast<uint64_t>(m >> 7) * col_tiles + (g >> 2);
+    return tile * 512u + (m & 31u) * 16u + ((m >> 5) & 3u) * 4u + (g & 3u);
+}
+
+// Store the UE8M0 byte of (row, group g) in the tiled plane; the last group's
+// lane also zeroes the padding groups of the row's last tile column.
+__device__ __forceinline__ void store_tiled(uint8_t *sc, uint32_t row, uint32_t g, uint32_t ng,
+                                            uint32_t e8) {
+    sc[tile128x4_offset(row, g, ng)] = static_cast<uint8_t>(e8);
+    if (g == ng - 1u)
+        for (uint32_t pad = ng; (pad & 3u) != 0u; ++pad) sc[tile128x4_offset(row, pad, ng)] = 0;
+}
 
 constexpr int kStripElems = 512;           // outputs per strip (32 lanes x 16)
 constexpr uint32_t kStripBytes = 1024;     // input bytes per strip (16-bit elements)
@@ -139,17 +155,29 @@ __device__ __forceinline__ void widen2<__half>(uint32_t w, float &lo, float &hi)
     hi = f.y;
 }
 
-// silu(g) * u in fp32, silu(g) = g * sigmoid(g).  With e = exp(-|g|) in (0, 1],
-// sigmoid(g) is 1/(1+e) for g >= 0 and e/(1+e) for g < 0, so neither the
-// exponential nor the reciprocal (of a value in [1, 2]) can overflow.  exp is
-// the hardware ex2 approximation and the reciprocal rcp.approx; the product
-// stays within a few fp32 ulps of silu(g) * u.
-__device__ __forceinline__ float silu_mul(float g, float u) {
-    const float e = __expf(-fabsf(g));
-    float r;
-    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(1.0f + e));
-    const float sig = g >= 0.0f ? r : e * r;
-    return g * sig * u;
+// silu(g) * u for a pair, in fp32: sigmoid(g) = 1 / (1 + 2^(-g * log2 e)) with
+// the hardware ex2 and rcp approximations, on packed f32x2 arithmetic where it
+// exists.  The extremes stay right without a branch: for g << 0 the power is
+// +inf (or the reciprocal flushes to zero) and silu is a zero of g's sign; for
+// g >> 0 the power flushes to 0 and sigmoid is 1.  The product stays within a
+// few fp32 ulps of silu(g) * u.
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float rcp_approx(float x) {
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float2 silu_mul2(float2 g, float2 u) {
+    constexpr float kNegLog2e = -1.4426950408889634f;
+    const float2 t = __fmul2_rn(g, make_float2(kNegLog2e, kNegLog2e));
+    const float2 d = __fadd2_rn(make_float2(ex2_approx(t.x), ex2_approx(t.y)),
+                                make_float2(1.0f, 1.0f));
+    const float2 sig = make_float2(rcp_approx(d.x), rcp_approx(d.y));
+    return __fmul2_rn(__fmul2_rn(g, sig), u);
 }
 
 // Packed pair of E4M3 codes: `lo` in bits 0-7, `hi` in bits 8-15.  Round to
@@ -524,8 +552,9 @@ __device__ __forceinline__ void quantize_strip(const uint32_t (&x)[8], const uin
             if constexpr (FUSED) {
                 float u0, u1;
                 widen2<In>(u[i], u0, u1);
-                v[2 * i] = silu_mul(v[2 * i], u0);
-                v[2 * i + 1] = silu_mul(v[2 * i + 1], u1);
+                const float2 y = silu_mul2(make_float2(v[2 * i], v[2 * i + 1]), make_float2(u0, u1));
+                v[2 * i] = y.x;
+                v[2 * i + 1] = y.y;
             }
         }
         float amax = 0.0f;
@@ -555,6 +584,8 @@ __device__ __forceinline__ void quantize_strip(const uint32_t (&x)[8], const uin
             if ((g & 3u) == 0u)
                 reinterpret_cast<uint32_t *>(sc)[static_cast<uint64_t>(g >> 2) * p.mpad + row] =
                     packed_word;
+        } else if (p.layout == kTiled128x4) {
+            store_tiled(sc, row, g, p.ng, gs.e8);
         } else {
             const uint64_t idx = (p.layout == kRowMajor) ? static_cast<uint64_t>(row) * p.ng + g
                                                          : static_cast<uint64_t>(g) * p.mpad + row;

@@ -79,8 +79,10 @@ __global__ void __launch_bounds__(kRowThreads)
                 if constexpr (FUSED) {
                     float u0, u1;
                     widen2<In>(u[j][i], u0, u1);
-                    v[j][2 * i] = silu_mul(v[j][2 * i], u0);
-                    v[j][2 * i + 1] = silu_mul(v[j][2 * i + 1], u1);
+                    const float2 y =
+                        silu_mul2(make_float2(v[j][2 * i], v[j][2 * i + 1]), make_float2(u0, u1));
+                    v[j][2 * i] = y.x;
+                    v[j][2 * i + 1] = y.y;
                 }
             }
 #pragma unroll
@@ -111,10 +113,13 @@ __global__ void __launch_bounds__(kRowThreads)
             }
             if (tid == 0) {
                 // one group per row: row-major, column-major and packed all put
-                // row r's scale at element / word r of the expert's plane
+                // row r's scale at element / word r of the expert's plane; the
+                // tiled layout has one tile column
                 uint8_t *sc = p.scales + sp.e * p.scale_expert_bytes;
                 if (p.layout == kPacked)
                     reinterpret_cast<uint32_t *>(sc)[row] = gs.e8;  // bytes 1..3 are 0
+                else if (p.layout == kTiled128x4)
+                    store_tiled(sc, row, 0u, 1u, gs.e8);
                 else if constexpr (KIND == Kind::E4M3_UE8M0)
                     sc[row] = static_cast<uint8_t>(gs.e8);
                 else

@@ -29,12 +29,13 @@ PQG_ERR_CUDA = -4
 
 PQG_BF16, PQG_FP16, PQG_E4M3, PQG_INT8 = 0, 1, 2, 3
 PQG_SCALE_FP32, PQG_SCALE_UE8M0 = 0, 1
-PQG_ROW_MAJOR, PQG_COL_MAJOR_TMA, PQG_UE8M0_PACKED = 0, 1, 2
+PQG_ROW_MAJOR, PQG_COL_MAJOR_TMA, PQG_UE8M0_PACKED, PQG_UE8M0_TILED_128x4 = 0, 1, 2, 3
 
 IN_DTYPES = {"bf16": PQG_BF16, "fp16": PQG_FP16}
 OUT_DTYPES = {"e4m3": PQG_E4M3, "int8": PQG_INT8}
 SCALE_FMTS = {"fp32": PQG_SCALE_FP32, "ue8m0": PQG_SCALE_UE8M0}
-LAYOUTS = {"row": PQG_ROW_MAJOR, "col": PQG_COL_MAJOR_TMA, "packed": PQG_UE8M0_PACKED}
+LAYOUTS = {"row": PQG_ROW_MAJOR, "col": PQG_COL_MAJOR_TMA, "packed": PQG_UE8M0_PACKED,
+           "tile128x4": PQG_UE8M0_TILED_128x4}
 
 EXPORTS = ("pqg_quant", "pqg_scales_bytes", "pqg_status_string", "pqg_last_cuda_error",
            "pqg_set_pdl", "pqg_launch_count", "pqg_version")
@@ -117,9 +118,10 @@ def scales_spec(M: int, K: int, group: int, scale_fmt: str = "fp32", layout: str
                 num_experts: int = 1):
     """(shape, torch dtype) of a contiguous scale buffer for these arguments.
 
-    row    : [E, M, ng]            fp32 or uint8
-    col    : [E, ng, M_pad]        fp32 or uint8
-    packed : [E, ceil(ng/4), M_pad] int32
+    row       : [E, M, ng]            fp32 or uint8
+    col       : [E, ng, M_pad]        fp32 or uint8
+    packed    : [E, ceil(ng/4), M_pad] int32
+    tile128x4 : [E, ceil(M/128) * ceil(ng/4) * 512] uint8
     """
     import torch
     nbytes = pqg_scales_bytes(num_experts, M, K, group, SCALE_FMTS[scale_fmt], LAYOUTS[layout])
@@ -130,6 +132,8 @@ def scales_spec(M: int, K: int, group: int, scale_fmt: str = "fp32", layout: str
         shape = (num_experts, M, ng)
     elif layout == "col":
         shape = (num_experts, ng, mpad)
+    elif layout == "tile128x4":
+        return (num_experts, (M + 127) // 128 * ((ng + 3) // 4) * 512), torch.uint8
     else:
         return (num_experts, (ng + 3) // 4, mpad), torch.int32
     return shape, (torch.uint8 if scale_fmt == "ue8m0" else torch.float32)

@@ -91,6 +91,14 @@ def _scale_planes(w, sbytes):
     matching UE8M0 byte table (or None)."""
     ng, mpad = w.K // w.group, (w.M + 3) // 4 * 4
     if w.scale_fmt == "ue8m0":
+        if w.layout == "tile128x4":
+            m = np.arange(w.M)[:, None]
+            g = np.arange(ng)[None, :]
+            off = (((m // 128) * ((ng + 3) // 4) + g // 4) * 512 + (m % 32) * 16
+                   + ((m % 128) // 32) * 4 + g % 4)
+            plane = sbytes.reshape(w.E, -1)
+            e8 = plane[:, off]
+            return np.exp2(e8.astype(np.float64) - 127.0), e8
         if w.layout == "packed":
             words = sbytes.reshape(w.E, (ng + 3) // 4, mpad, 4)
             e8 = words.transpose(0, 2, 1, 3).reshape(w.E, mpad, -1)[:, :w.M, :ng]
@@ -127,7 +135,12 @@ def check_fused(w, *, max_flip_frac=1e-4, rel_tol=7e-2, **kw):
     # scale bytes outside live (row, group) cells must be untouched
     ng, mpad = K // G, (M + 3) // 4 * 4
     idx = np.arange(gs.size)
-    if w.layout == "packed":
+    if w.layout == "tile128x4":
+        plane = (M + 127) // 128 * ((ng + 3) // 4) * 512
+        e_of, off = idx // plane, idx % plane
+        tile, inner = off // 512, off % 512
+        m_of = (tile // ((ng + 3) // 4)) * 128 + ((inner // 4) % 4) * 32 + inner // 16
+    elif w.layout == "packed":
         word = idx // 4
         m_of, e_of = word % mpad, word // (((ng + 3) // 4) * mpad)
     else:

@@ -80,7 +80,7 @@ def test_enum_values_match_header():
     for name in ("PQG_OK", "PQG_ERR_INVALID_ARG", "PQG_ERR_UNSUPPORTED", "PQG_ERR_ALIGNMENT",
                  "PQG_ERR_CUDA", "PQG_BF16", "PQG_FP16", "PQG_E4M3", "PQG_INT8",
                  "PQG_SCALE_FP32", "PQG_SCALE_UE8M0", "PQG_ROW_MAJOR", "PQG_COL_MAJOR_TMA",
-                 "PQG_UE8M0_PACKED"):
+                 "PQG_UE8M0_PACKED", "PQG_UE8M0_TILED_128x4"):
         m = re.search(rf"\b{name}\s*=\s*(-?\d+)", text)
         assert m and int(m.group(1)) == getattr(pqg, name), name
 
@@ -98,7 +98,8 @@ def test_pdl_toggle_round_trips():
 @pytest.mark.parametrize("E,M,K,G", [(1, 4, 256, 128), (1, 8192, 7168, 128), (3, 5, 640, 64),
                                      (32, 2048, 2048, 128), (2, 1, 96, 32), (1, 0, 128, 128)])
 @pytest.mark.parametrize("fmt,layout", [("fp32", "row"), ("fp32", "col"), ("ue8m0", "row"),
-                                        ("ue8m0", "col"), ("ue8m0", "packed")])
+                                        ("ue8m0", "col"), ("ue8m0", "packed"),
+                                        ("ue8m0", "tile128x4")])
 def test_scales_bytes_matches_oracle(E, M, K, G, fmt, layout):
     import oracle
     lib = oracle.load()
@@ -163,6 +164,8 @@ def call(**kw):
     (dict(num_experts=4096, M=1 << 12, K=1 << 14), pqg.PQG_ERR_INVALID_ARG),  # 2^31 strips
     (dict(out_dtype=pqg.PQG_INT8, scale_fmt=pqg.PQG_SCALE_UE8M0), pqg.PQG_ERR_UNSUPPORTED),
     (dict(scale_layout=pqg.PQG_UE8M0_PACKED), pqg.PQG_ERR_UNSUPPORTED),
+    (dict(scale_layout=pqg.PQG_UE8M0_TILED_128x4), pqg.PQG_ERR_UNSUPPORTED),
+    (dict(scale_layout=4), pqg.PQG_ERR_INVALID_ARG),
     (dict(in_ptr=0), pqg.PQG_ERR_INVALID_ARG),
     (dict(out_ptr=0), pqg.PQG_ERR_INVALID_ARG),
     (dict(scales_ptr=0), pqg.PQG_ERR_INVALID_ARG),

@@ -39,6 +39,7 @@ MUTANTS = {
     "packed_padding_not_zeroed": ("((uint8_t *)scales)[word * 4 + b] = 0;", ";"),
     "fp16_subnormal_exponent": ("v = ldexp((double)m, -24);", "v = ldexp((double)m, -25);"),
     "int8_truncates": ("double n = nearbyint((double)t);", "double n = trunc((double)t);"),
+    "tile_rows_not_interleaved": ("(r % 32) * 16 + (r / 32) * 4", "(r % 32) * 4 + (r / 32) * 128"),
 }
 
 

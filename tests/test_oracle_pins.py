@@ -409,6 +409,32 @@ def test_scale_layouts_are_one_table():
     assert np.array_equal(s_f.reshape(5, 8)[:, :M], s_g.reshape(M, 5).T)
 
 
+def test_tile128x4_layout_positions():
+    """The 128x4 tiled UE8M0 layout (MXFP8 producer): bytes at hand-derived
+    positions, padding columns 0, padding rows untouched."""
+    M, K, G = 130, 5 * 32, 32            # 2 row tiles (ragged), ng = 5 -> 2 column tiles
+    x = inputs.bf16_bits(inputs.normal((1, M, K), 24) * 3)
+    _, row = oracle.quant(x, M=M, K=K, group=G, scale_fmt="ue8m0", layout="row")
+    _, til = oracle.quant(x, M=M, K=K, group=G, scale_fmt="ue8m0", layout="tile128x4")
+    row = row.reshape(M, 5)
+    til = til.reshape(-1)
+    assert til.size == 2 * 2 * 512
+    # (m, g) -> byte, worked by hand: tile = (m // 128) * 2 + g // 4, then
+    # (m % 32) * 16 + ((m % 128) // 32) * 4 + g % 4 inside the tile
+    for (m, g), byte in {(0, 0): 0, (1, 0): 16, (32, 0): 4, (33, 1): 21, (127, 3): 511,
+                         (0, 4): 512, (128, 0): 1024, (129, 4): 1552, (129, 0): 1040}.items():
+        assert int(til[byte]) == int(row[m, g]), (m, g, byte)
+    # padding columns (g = 5..7) of quantized rows are 0; padding rows untouched
+    for m in (0, 77, 129):
+        for g in (5, 6, 7):
+            tile = (m // 128) * 2 + g // 4
+            byte = tile * 512 + (m % 32) * 16 + ((m % 128) // 32) * 4 + g % 4
+            assert til[byte] == 0
+    assert til[1024 + 2 * 16] == 0xA5                        # row 130: a padding row
+    # every quantized exponent appears once
+    assert sorted(til[til != 0xA5].tolist()) == sorted(row.reshape(-1).tolist() + [0] * (3 * M))
+
+
 def test_masked_rows_untouched_and_full_mask_equals_flat():
     E, M, K = 3, 8, 256
     x = inputs.bf16_bits(inputs.normal((E, M, 2 * K), 22))

@@ -18,6 +18,7 @@ pytestmark = pytest.mark.gpu
 KINDS = [  # (out_dtype, scale_fmt, layout)
     ("e4m3", "fp32", "row"), ("e4m3", "fp32", "col"),
     ("e4m3", "ue8m0", "row"), ("e4m3", "ue8m0", "col"), ("e4m3", "ue8m0", "packed"),
+    ("e4m3", "ue8m0", "tile128x4"),
     ("int8", "fp32", "row"), ("int8", "fp32", "col"),
 ]
 
@@ -304,3 +305,36 @@ def test_per_token_fused_and_masked(K):
 def test_per_token_full_size():
     w = inputs.flat_hidden(layout="row", scale_fmt="fp32").with_(group=7168)
     check_exact(w)
+
+
+# --------------------------------------------------------------------------
+# grouped-contiguous (varlen) tokens: a flat call over the packed rows
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("kind", [("e4m3", "ue8m0", "row"), ("e4m3", "fp32", "row")],
+                         ids=lambda k: "_".join(k))
+def test_varlen_contiguous_equals_masked(kind):
+    """The tokens of each expert packed back to back (blocks padded to 128 rows,
+    as a grouped-contiguous GEMM takes them) quantize, with one flat fused call,
+    to the same bytes as masked dispatch over [E, M_max, 2K]."""
+    E, M_max, K = 4, 256, 1024
+    counts = np.array([100, 0, 256, 37], np.int32)
+    w = make(M_max, K, 128, kind, fused=True, E=E, seed=41, masked_m=counts, expected_m=100)
+    mq, ms = run_gpu(w)
+    mq = mq.reshape(E, M_max, K)
+    ms = ms.view(np.float32 if kind[1] == "fp32" else np.uint8).reshape(E, M_max, K // 128)
+    blocks = [(-(-int(c) // 128)) * 128 for c in counts]
+    packed = np.zeros((1, sum(blocks), 2 * K), np.uint16)
+    off = np.concatenate([[0], np.cumsum(blocks)])
+    for e in range(E):
+        packed[0, off[e]:off[e] + counts[e]] = w.x[e, :counts[e]]
+    flat = inputs.Workload("varlen", packed, M=sum(blocks), K=K, group=128, out_dtype=kind[0],
+                           scale_fmt=kind[1], layout="row", fused=True)
+    fq, fs = run_gpu(flat)
+    fq = fq.reshape(-1, K)
+    fs = fs.view(np.float32 if kind[1] == "fp32" else np.uint8).reshape(-1, K // 128)
+    for e in range(E):
+        n = int(counts[e])
+        assert_same(fq[off[e]:off[e] + n].reshape(-1), mq[e, :n].reshape(-1), f"codes e={e}")
+        assert_same(fs[off[e]:off[e] + n].view(np.uint8).reshape(-1),
+                    ms[e, :n].view(np.uint8).reshape(-1), f"scales e={e}")

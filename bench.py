@@ -51,6 +51,7 @@ def workloads():
         "flat_hidden_fp32": lambda: inputs.flat_hidden(layout="row", scale_fmt="fp32"),
         "per_token": lambda: inputs.flat_hidden(layout="row", scale_fmt="fp32").with_(
             group=7168, name="per_token_8192x7168"),
+        "mxfp4": lambda: inputs.mxfp4(),
         "fused": lambda: inputs.fused(),
         "masked": lambda: inputs.masked(),
         "masked_decode": lambda: inputs.masked(decode=True),
@@ -65,7 +66,7 @@ def describe(w) -> dict:
         [w.M, 2 * w.K if w.fused else w.K]
     d = {"workload": w.name, "input_shape": shape, "in_dtype": w.in_dtype,
          "out_dtype": w.out_dtype, "group": w.group,
-         "scales": f"{w.scale_fmt} {dict(row='row-major', col='column-major TMA-aligned', packed='UE8M0-packed column-major')[w.layout]}",
+         "scales": f"{w.scale_fmt} {dict(row='row-major', col='column-major TMA-aligned', packed='UE8M0-packed column-major', tile128x4='128x4 tiled (MX)')[w.layout]}",
          "fused_silu_mul": w.fused, "rows_quantized": w.rows,
          "algorithmic_bytes_per_step": w.algorithmic_bytes()}
     if w.masked_m is not None:
@@ -262,7 +263,7 @@ def run_ours(args, w, rank: int, world: int, local_rank: int) -> dict | None:
     x0 = torch.from_numpy(np.ascontiguousarray(w.x).view(np.int16)).view(dt).to(dev)
     nbytes = pqg.pqg_scales_bytes(w.E, w.M, w.K, w.group, pqg.SCALE_FMTS[w.scale_fmt],
                                   pqg.LAYOUTS[w.layout])
-    n_out = w.E * w.M * w.K
+    n_out = w.E * w.M * (w.K // 2 if w.out_dtype == "e2m1" else w.K)
     footprint = x0.numel() * 2 + n_out + nbytes
     sets = max(1, min(8, -(-4 * L2_BYTES // footprint)))
     xs = [x0] + [x0.clone() for _ in range(sets - 1)]
@@ -372,7 +373,7 @@ def latency_m1(w, dev, stream) -> dict:
     x = torch.zeros((1, width), dtype=torch.bfloat16 if w.in_dtype == "bf16" else torch.float16,
                     device=dev)
     x.normal_()
-    out = torch.empty(w.K, dtype=torch.uint8, device=dev)
+    out = torch.empty(w.K // 2 if w.out_dtype == "e2m1" else w.K, dtype=torch.uint8, device=dev)
     nb = pqg.pqg_scales_bytes(1, 1, w.K, w.group, pqg.SCALE_FMTS[w.scale_fmt],
                               pqg.LAYOUTS[w.layout])
     sc = torch.empty(nb, dtype=torch.uint8, device=dev)

@@ -80,7 +80,9 @@ enum pqg_dtype {
     PQG_BF16 = 0, /* input: bfloat16                                  */
     PQG_FP16 = 1, /* input: IEEE binary16                             */
     PQG_E4M3 = 2, /* output: OCP FP8 E4M3 "fn" (max 448, no inf)       */
-    PQG_INT8 = 3  /* output: two's-complement int8                    */
+    PQG_INT8 = 3, /* output: two's-complement int8                    */
+    PQG_E2M1 = 4  /* output: OCP FP4 E2M1 (max 6), two codes per byte,
+                     element 2i in bits 0-3 and 2i+1 in bits 4-7 (MXFP4) */
 };
 
 /* Scale formats. */
@@ -125,8 +127,8 @@ enum pqg_scale_layout {
  * in       device, read-only.  [num_experts][M][K] elements of in_dtype, or
  *          [num_experts][M][2K] when fuse_silu_mul (row = gate | up).  Rows are
  *          dense (row stride = K or 2K elements).  32-byte aligned.
- * out      device.  [num_experts][M][K] one-byte codes (E4M3 or INT8).
- *          16-byte aligned.
+ * out      device.  [num_experts][M][K] one-byte codes (E4M3 or INT8), or
+ *          [num_experts][M][K/2] bytes of E2M1 code pairs.  16-byte aligned.
  * scales   device.  pqg_scales_bytes(num_experts, M, K, group, scale_fmt,
  *          scale_layout) bytes in the chosen layout.  4-byte aligned for fp32
  *          scales and packed words, any alignment for UE8M0 bytes.
@@ -138,8 +140,11 @@ enum pqg_scale_layout {
  * group    G in {32, 64, 128}, or G == K for one scale per row (per-token
  *          quantization, as tf_per_token_quant_fp8 on the TeleFuser page;
  *          K a multiple of 16, at most 16384).
- * in_dtype PQG_BF16 or PQG_FP16.   out_dtype PQG_E4M3 or PQG_INT8.
- * scale_fmt, scale_layout   see above.  PQG_SCALE_UE8M0 requires PQG_E4M3, and
+ * in_dtype PQG_BF16 or PQG_FP16.   out_dtype PQG_E4M3, PQG_INT8 or PQG_E2M1.
+ *          PQG_E2M1 (MXFP4: "block_size = 32 -> MXFP4" in the FlashInfer notes,
+ *          section 6) needs PQG_SCALE_UE8M0 and G in {32, 64, 128}; its scale
+ *          is 2^ceil(log2(amax / 6)) by the same bit rule with FMAX = 6.
+ * scale_fmt, scale_layout   see above.  PQG_SCALE_UE8M0 rejects PQG_INT8, and
  *          PQG_UE8M0_PACKED and PQG_UE8M0_TILED_128x4 require PQG_SCALE_UE8M0
  *          (else PQG_ERR_UNSUPPORTED).
  * fuse_silu_mul  nonzero: quantize silu(gate) * up (see the numerics above).

@@ -31,6 +31,7 @@ _LOCK = threading.Lock()
 _lib = None
 
 LAYOUTS = {"row": 0, "col": 1, "packed": 2, "tile128x4": 3}
+OUT_KINDS = {"e4m3": 0, "int8": 1, "e2m1": 2}
 
 
 def build(force: bool = False, src: str = _SRC, out: str = _LIB_PATH) -> str:
@@ -83,7 +84,7 @@ def load(path: str | None = None):
         lib.pqgo_int8_encode.restype = ctypes.c_int8
         lib.pqgo_int8_encode.argtypes = [f32]
         for name in ("pqgo_decode_n", "pqgo_e4m3_encode_n", "pqgo_int8_encode_n",
-                     "pqgo_ue8m0_exponent_n"):
+                     "pqgo_ue8m0_exponent_n", "pqgo_e2m1_encode_n", "pqgo_ue8m0_exponent_fmax_n"):
             getattr(lib, name).restype = None
         lib.pqgo_decode_n.argtypes = [vp, vp, i64, i32]
         lib.pqgo_silu_mul_n.restype = None
@@ -91,6 +92,8 @@ def load(path: str | None = None):
         lib.pqgo_e4m3_encode_n.argtypes = [vp, vp, i64]
         lib.pqgo_int8_encode_n.argtypes = [vp, vp, i64]
         lib.pqgo_ue8m0_exponent_n.argtypes = [vp, vp, i64]
+        lib.pqgo_e2m1_encode_n.argtypes = [vp, vp, i64]
+        lib.pqgo_ue8m0_exponent_fmax_n.argtypes = [vp, vp, i64, f32]
         lib.pqgo_scale_fp32_n.restype = None
         lib.pqgo_scale_fp32_n.argtypes = [vp, vp, i64, i32]
         if default:
@@ -140,6 +143,22 @@ def int8_encode(t, lib=None) -> np.ndarray:
     q = np.empty(t.shape, np.int8)
     lib.pqgo_int8_encode_n(_ptr(t), _ptr(q), t.size)
     return q
+
+
+def e2m1_encode(t, lib=None) -> np.ndarray:
+    lib = lib or load()
+    t = _c(t, np.float32)
+    q = np.empty(t.shape, np.uint8)
+    lib.pqgo_e2m1_encode_n(_ptr(t), _ptr(q), t.size)
+    return q
+
+
+def ue8m0_exponent_fmax(amax, fmax: float, lib=None) -> np.ndarray:
+    lib = lib or load()
+    a = _c(amax, np.float32)
+    e = np.empty(a.shape, np.uint8)
+    lib.pqgo_ue8m0_exponent_fmax_n(_ptr(a), _ptr(e), a.size, float(fmax))
+    return e
 
 
 def ue8m0_exponent(amax, lib=None) -> np.ndarray:
@@ -193,22 +212,23 @@ def quant(x_bits, *, M: int, K: int, group: int, E: int = 1, in_dtype: str = "bf
     the E axis may be omitted when E == 1).  ``out``/``scales`` may be given
     prefilled (rows the call must not touch are then checked by the caller);
     otherwise they are allocated filled with ``fill``.  Returns (out, scales)
-    shaped [E, M, K] and per ``scales_shape``.
+    shaped [E, M, K] ([E, M, K/2] for E2M1) and per ``scales_shape``.
     """
     lib = lib or load()
     x = _c(x_bits, np.uint16)
     width = 2 * K if fused else K
     if x.size != E * M * width:
         raise ValueError(f"x has {x.size} elements, expected {E * M * width}")
+    kbytes = K // 2 if out_dtype == "e2m1" else K
     if out is None:
-        out = np.full((E, M, K), fill, np.uint8)
+        out = np.full((E, M, kbytes), fill, np.uint8)
     shape, sdt = scales_shape(E, M, K, group, scale_fmt, layout)
     if scales is None:
         scales = np.empty(shape, sdt)
         scales.view(np.uint8).fill(fill)
     nbytes = lib.pqgo_scales_nbytes(E, M, K, group, int(scale_fmt == "ue8m0"),
                                     LAYOUTS[layout])
-    if scales.nbytes != nbytes or out.size != E * M * K:
+    if scales.nbytes != nbytes or out.size != E * M * kbytes:
         raise ValueError("output buffers have the wrong size")
     mm = None
     if masked_m is not None:
@@ -216,7 +236,7 @@ def quant(x_bits, *, M: int, K: int, group: int, E: int = 1, in_dtype: str = "bf
         if mm.size != E:
             raise ValueError("masked_m needs one entry per expert")
     rc = lib.pqgo_quant(_ptr(x), _ptr(out), _ptr(scales), E, M, K, group,
-                        int(in_dtype == "fp16"), int(out_dtype == "int8"),
+                        int(in_dtype == "fp16"), OUT_KINDS[out_dtype],
                         int(scale_fmt == "ue8m0"), LAYOUTS[layout], int(bool(fused)),
                         None if mm is None else _ptr(mm))
     if rc != 0:

@@ -36,6 +36,9 @@
  *     it is never rounded to the input dtype.
  *   - every rounding is to nearest, ties to even; E4M3 is the OCP "fn"
  *     variant (no infinities, 448 largest finite), zero keeps the sign of t.
+ *   - FP4 (MXFP4, the FlashInfer notes' "block_size = 32 -> MXFP4"): OCP E2M1
+ *     codes (largest magnitude 6), UE8M0 scales by the same rule with FMAX = 6,
+ *     two codes per byte with element 2i in bits 0-3 and 2i+1 in bits 4-7.
  *   - column-major layouts pad the row count to a multiple of 4 (16 bytes of
  *     fp32 or one int32 word per 4 rows), padding rows are never written.
  *   - the UE8M0-packed layout stores the exponents of groups 4j..4j+3 of a
@@ -62,9 +65,12 @@
 /* ---- constants of the method (values, not code, shared with nobody) ---- */
 #define PQGO_FMAX_E4M3 448.0f   /* largest finite E4M3 value ([PR] FMAX)       */
 #define PQGO_FMAX_INT8 127.0f   /* INT8 scale divisor ([PR] ref_int8)          */
+#define PQGO_FMAX_E2M1 6.0f     /* largest finite OCP E2M1 value (MXFP4)       */
 #define PQGO_EPS 1e-10f         /* absmax floor ([PR] "不低于 EPS")             */
 
-/* layouts understood by the oracle (numbered for the Python wrapper) */
+/* output kinds and layouts understood by the oracle (numbered for the Python
+ * wrapper) */
+enum { PQGO_OUT_E4M3 = 0, PQGO_OUT_INT8 = 1, PQGO_OUT_E2M1 = 2 };
 enum { PQGO_ROW = 0, PQGO_COL = 1, PQGO_PACKED = 2, PQGO_TILE128X4 = 3 };
 
 /* ------------------------------------------------------------------------ */
@@ -134,14 +140,16 @@ float pqgo_scale_fp32(float amax, int out_int8) {
  * raw = amax / FMAX in fp32; take raw's biased exponent field; add one when
  * raw's 23-bit mantissa is nonzero (rounds the scale up to a power of two).
  * The scale is 2^(byte - 127). */
-int pqgo_ue8m0_exponent(float amax) {
-    float raw = amax / PQGO_FMAX_E4M3;
+int pqgo_ue8m0_exponent_fmax(float amax, float fmax) {
+    float raw = amax / fmax;
     uint32_t bits;
     memcpy(&bits, &raw, sizeof bits);
     int biased = (int)((bits >> 23) & 0xFF);
     int bump = (bits & 0x7FFFFF) != 0;
     return biased + bump;
 }
+
+int pqgo_ue8m0_exponent(float amax) { return pqgo_ue8m0_exponent_fmax(amax, PQGO_FMAX_E4M3); }
 
 /* ------------------------------------------------------------------------ */
 /* Output encoders                                                           */
@@ -183,6 +191,28 @@ int8_t pqgo_int8_encode(float t) {
     return (int8_t)n;
 }
 
+/* Saturating cast to OCP FP4 E2M1: sign bit, 2 exponent bits (bias 1), 1
+ * mantissa bit.  Normal values (1 + m/2) * 2^(e - 1) for e = 1..3, subnormal
+ * m * 0.5; the magnitudes are 0, 0.5, 1, 1.5, 2, 3, 4, 6.  |t| is clamped to
+ * 6, then rounded to the nearest magnitude with ties to an even mantissa; a
+ * value that rounds to zero keeps the sign of t.  Returns the 4-bit code. */
+uint8_t pqgo_e2m1_encode(float t) {
+    uint8_t sign = signbit(t) ? 0x8 : 0x0;
+    double a = fabs((double)t);
+    if (a > 6.0) a = 6.0;
+    int E = (a >= 1.0) ? ilogb(a) : 0;      /* binade; below 1 the spacing is 0.5 */
+    double quantum = ldexp(1.0, E - 1);
+    double n = nearbyint(a / quantum);        /* ties to even */
+    double r = n * quantum;
+    if (r == 0.0) return sign;
+    if (r < 1.0) return (uint8_t)(sign | 0x1); /* 0.5: subnormal */
+    {
+        int Er = ilogb(r);
+        int mant = (int)(r / ldexp(1.0, Er - 1)) - 2;
+        return (uint8_t)(sign | ((Er + 1) << 1) | mant);
+    }
+}
+
 /* ------------------------------------------------------------------------ */
 /* Scale layouts                                                             */
 /* ------------------------------------------------------------------------ */
@@ -217,17 +247,22 @@ int64_t pqgo_scales_nbytes(int64_t E, int64_t M, int64_t K, int G,
 /* Quantize E experts of M rows (E = 1, masked_m = NULL: flat dispatch).
  *   in      : [E][M][K] (or [E][M][2K] when fused: gate | up), raw 16-bit
  *             bf16 or fp16 patterns
- *   out     : [E][M][K] one code byte per element
+ *   out     : [E][M][K] one code byte per element ([E][M][K/2] for E2M1, two
+ *             codes per byte)
  *   scales  : layout-dependent (see pqgo_scales_nbytes)
  *   masked_m: host array of E row counts, or NULL.  Rows m >= masked_m[e]
  *             (clamped to [0, M]) are not touched; neither are padding rows.
  * Returns 0, -1 for an invalid argument, -2 for a non-finite input value. */
 int pqgo_quant(const uint16_t *in, uint8_t *out, void *scales, int64_t E,
-               int64_t M, int64_t K, int G, int in_fp16, int out_int8,
+               int64_t M, int64_t K, int G, int in_fp16, int out_kind,
                int scale_ue8m0, int layout, int fused,
                const int32_t *masked_m) {
+    const int out_int8 = out_kind == PQGO_OUT_INT8;
+    const int out_e2m1 = out_kind == PQGO_OUT_E2M1;
     if (E < 1 || M < 0 || K <= 0 || G <= 0 || K % G != 0) return -1;
     if (layout < PQGO_ROW || layout > PQGO_TILE128X4) return -1;
+    if (out_kind < PQGO_OUT_E4M3 || out_kind > PQGO_OUT_E2M1) return -1;
+    if (out_e2m1 && (!scale_ue8m0 || G % 2 != 0)) return -1;  /* MXFP4: UE8M0 */
     if (scale_ue8m0 && out_int8) return -1;       /* UE8M0 pairs with FMAX */
     if ((layout == PQGO_PACKED || layout == PQGO_TILE128X4) && !scale_ue8m0) return -1;
 
@@ -247,7 +282,7 @@ int pqgo_quant(const uint16_t *in, uint8_t *out, void *scales, int64_t E,
         }
         for (int64_t m = 0; m < rows && status == 0; ++m) {
             const uint16_t *xrow = in + (e * M + m) * in_width;
-            uint8_t *qrow = out + (e * M + m) * K;
+            uint8_t *qrow = out + (e * M + m) * (out_e2m1 ? K / 2 : K);
             for (int64_t g = 0; g < ng; ++g) {
                 /* 1. decode (and fuse) the G values of this group */
                 for (int i = 0; i < G; ++i) {
@@ -267,7 +302,8 @@ int pqgo_quant(const uint16_t *in, uint8_t *out, void *scales, int64_t E,
                 float s;
                 int ebyte = 0;
                 if (scale_ue8m0) {
-                    ebyte = pqgo_ue8m0_exponent(amax);
+                    ebyte = pqgo_ue8m0_exponent_fmax(amax, out_e2m1 ? PQGO_FMAX_E2M1
+                                                                    : PQGO_FMAX_E4M3);
                     s = ldexpf(1.0f, ebyte - 127);
                 } else {
                     s = pqgo_scale_fp32(amax, out_int8);
@@ -276,8 +312,17 @@ int pqgo_quant(const uint16_t *in, uint8_t *out, void *scales, int64_t E,
                 /* 4. codes: saturating cast of x / s */
                 for (int i = 0; i < G; ++i) {
                     float t = v[i] / s;
-                    qrow[g * G + i] = out_int8 ? (uint8_t)pqgo_int8_encode(t)
-                                               : pqgo_e4m3_encode(t);
+                    if (out_e2m1) {
+                        int64_t j = g * G + i;
+                        uint8_t code = pqgo_e2m1_encode(t);
+                        if (j % 2 == 0)
+                            qrow[j / 2] = code;                       /* low nibble  */
+                        else
+                            qrow[j / 2] = (uint8_t)(qrow[j / 2] | (code << 4)); /* high */
+                    } else {
+                        qrow[g * G + i] = out_int8 ? (uint8_t)pqgo_int8_encode(t)
+                                                   : pqgo_e4m3_encode(t);
+                    }
                 }
 
                 /* 5. scale store */
@@ -331,6 +376,14 @@ void pqgo_silu_mul_n(const float *gate, const float *up, float *y, int64_t n) {
 
 void pqgo_e4m3_encode_n(const float *t, uint8_t *q, int64_t n) {
     for (int64_t i = 0; i < n; ++i) q[i] = pqgo_e4m3_encode(t[i]);
+}
+
+void pqgo_e2m1_encode_n(const float *t, uint8_t *q, int64_t n) {
+    for (int64_t i = 0; i < n; ++i) q[i] = pqgo_e2m1_encode(t[i]);
+}
+
+void pqgo_ue8m0_exponent_fmax_n(const float *amax, uint8_t *e, int64_t n, float fmax) {
+    for (int64_t i = 0; i < n; ++i) e[i] = (uint8_t)pqgo_ue8m0_exponent_fmax(amax[i], fmax);
 }
 
 void pqgo_int8_encode_n(const float *t, int8_t *q, int64_t n) {

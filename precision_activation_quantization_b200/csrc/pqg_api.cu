@@ -101,11 +101,15 @@ int pqg_quant(const void *in, void *out, void *scales, int64_t M, int64_t num_ex
               int fuse_silu_mul, const int32_t *masked_m, int64_t expected_m,
               pqg_stream_t stream) {
     if (in_dtype != PQG_BF16 && in_dtype != PQG_FP16) return PQG_ERR_INVALID_ARG;
-    if (out_dtype != PQG_E4M3 && out_dtype != PQG_INT8) return PQG_ERR_INVALID_ARG;
+    if (out_dtype != PQG_E4M3 && out_dtype != PQG_INT8 && out_dtype != PQG_E2M1)
+        return PQG_ERR_INVALID_ARG;
     int64_t plane = 0;
     const int st = check_geometry(num_experts, M, K, group, scale_fmt, scale_layout, &plane);
     if (st != PQG_OK) return st;
-    if (scale_fmt == PQG_SCALE_UE8M0 && out_dtype != PQG_E4M3) return PQG_ERR_UNSUPPORTED;
+    if (scale_fmt == PQG_SCALE_UE8M0 && out_dtype == PQG_INT8) return PQG_ERR_UNSUPPORTED;
+    if (out_dtype == PQG_E2M1 &&
+        (scale_fmt != PQG_SCALE_UE8M0 || (group != 32 && group != 64 && group != 128)))
+        return PQG_ERR_UNSUPPORTED;  // MXFP4: UE8M0 scales, groups of 32/64/128
     if (M == 0) return PQG_OK;
 
     if (in == nullptr || out == nullptr || scales == nullptr) return PQG_ERR_INVALID_ARG;
@@ -117,7 +121,8 @@ int pqg_quant(const void *in, void *out, void *scales, int64_t M, int64_t num_ex
 
     const int64_t in_row_bytes = K * 2 * (fuse_silu_mul ? 2 : 1);
     const int64_t in_bytes = num_experts * M * in_row_bytes;
-    const int64_t out_bytes = num_experts * M * K;
+    const int64_t out_row_bytes = out_dtype == PQG_E2M1 ? K / 2 : K;
+    const int64_t out_bytes = num_experts * M * out_row_bytes;
     if (overlaps(in, in_bytes, out, out_bytes) || overlaps(in, in_bytes, scales, plane * num_experts) ||
         overlaps(out, out_bytes, scales, plane * num_experts))
         return PQG_ERR_INVALID_ARG;
@@ -128,7 +133,8 @@ int pqg_quant(const void *in, void *out, void *scales, int64_t M, int64_t num_ex
     a.p.scales = static_cast<uint8_t *>(scales);
     a.p.masked_m = masked_m;
     a.p.in_expert_bytes = M * in_row_bytes;
-    a.p.out_expert_bytes = M * K;
+    a.p.out_expert_bytes = M * out_row_bytes;
+    a.p.out_row_bytes = static_cast<uint32_t>(out_row_bytes);
     a.p.scale_expert_bytes = plane;
     a.p.M = static_cast<uint32_t>(M);
     a.p.K = static_cast<uint32_t>(K);
@@ -143,9 +149,10 @@ int pqg_quant(const void *in, void *out, void *scales, int64_t M, int64_t num_ex
     a.expected_strips = static_cast<uint64_t>(num_experts * grid_rows) * a.p.segs;
     a.expected_rows = static_cast<uint64_t>(num_experts * grid_rows);
     a.group = group;
-    a.kind = scale_fmt == PQG_SCALE_UE8M0 ? pqg::Kind::E4M3_UE8M0
-             : out_dtype == PQG_INT8      ? pqg::Kind::INT8_FP32
-                                          : pqg::Kind::E4M3_FP32;
+    a.kind = out_dtype == PQG_E2M1           ? pqg::Kind::E2M1_UE8M0
+             : scale_fmt == PQG_SCALE_UE8M0 ? pqg::Kind::E4M3_UE8M0
+             : out_dtype == PQG_INT8        ? pqg::Kind::INT8_FP32
+                                            : pqg::Kind::E4M3_FP32;
     a.fused = fuse_silu_mul != 0;
     a.pdl = g_pdl.load(std::memory_order_relaxed) != 0;
     a.stream = reinterpret_cast<cudaStream_t>(stream);

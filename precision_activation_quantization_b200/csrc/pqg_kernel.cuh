@@ -53,7 +53,12 @@
 
 namespace pqg {
 
-enum class Kind : int { E4M3_FP32 = 0, E4M3_UE8M0 = 1, INT8_FP32 = 2 };
+enum class Kind : int { E4M3_FP32 = 0, E4M3_UE8M0 = 1, INT8_FP32 = 2, E2M1_UE8M0 = 3 };
+
+// Kinds whose scale is a UE8M0 power of two.
+__host__ __device__ constexpr bool is_ue8m0(Kind k) {
+    return k == Kind::E4M3_UE8M0 || k == Kind::E2M1_UE8M0;
+}
 
 // Runtime scale layouts (same numbering as the C ABI's pqg_scale_layout).
 enum : uint32_t { kRowMajor = 0, kColMajor = 1, kPacked = 2, kTiled128x4 = 3 };
@@ -84,11 +89,12 @@ struct Params {
     uint8_t *scales;           // expert 0's scale plane (byte address)
     const int32_t *masked_m;   // device int32[experts], or null: all M rows
     int64_t in_expert_bytes;   // M * in_row_bytes
-    int64_t out_expert_bytes;  // M * K
+    int64_t out_expert_bytes;  // M * out_row_bytes
     int64_t scale_expert_bytes;
     uint32_t M;                // rows per expert (capacity when masked)
     uint32_t K;                // outputs per row
     uint32_t in_row_bytes;     // 2K (plain) or 4K (fused), in bytes
+    uint32_t out_row_bytes;    // K (one byte per code) or K/2 (E2M1, two per byte)
     uint32_t ng;               // groups per row
     uint32_t segs;             // strips per row = ceil(K / 512)
     uint32_t mpad;             // rows of a column-major plane (M rounded up to 4)
@@ -117,6 +123,10 @@ __device__ __forceinline__ void load32B(const void *p, uint32_t (&r)[8]) {
         : "l"(p));
 }
 
+__device__ __forceinline__ void store8B(void *p, uint32_t a, uint32_t b) {
+    asm volatile("st.global.v2.b32 [%0], {%1,%2};" ::"l"(p), "r"(a), "r"(b) : "memory");
+}
+
 __device__ __forceinline__ void store16B(void *p, uint32_t a, uint32_t b, uint32_t c,
                                          uint32_t d) {
     asm volatile("st.global.v4.b32 [%0], {%1,%2,%3,%4};" ::"l"(p), "r"(a), "r"(b), "r"(c),
@@ -125,9 +135,19 @@ __device__ __forceinline__ void store16B(void *p, uint32_t a, uint32_t b, uint32
 }
 
 // Programmatic dependent launch: wait for the preceding grid's memory before the
-// first global access; let the next grid start its prologue when we are done.
+// first global access; let the next grid start its prologue when we are done
+// (or, with PQG_EARLY_TRIGGER, as soon as every CTA has started).
+#ifndef PQG_EARLY_TRIGGER
+#define PQG_EARLY_TRIGGER 0
+#endif
 __device__ __forceinline__ void wait_for_producer() {
     asm volatile("griddepcontrol.wait;" ::: "memory");
+#if PQG_EARLY_TRIGGER
+    // A dependent grid launches only once every CTA of this grid has signalled
+    // (or exited), so signalling at entry cannot starve this grid of SMs; the
+    // dependent's own griddepcontrol.wait still waits for this grid to finish.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+#endif
 }
 __device__ __forceinline__ void release_dependents() {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -185,6 +205,16 @@ __device__ __forceinline__ float2 silu_mul2(float2 g, float2 u) {
 __device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
     uint16_t r;
     asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// Packed pair of OCP E2M1 codes: `lo` in bits 0-3, `hi` in bits 4-7.  Round to
+// nearest even; satfinite clamps to +-6 (never reached: |t| <= 6 here).
+__device__ __forceinline__ uint32_t e2m1x2(float lo, float hi) {
+    uint32_t r;
+    asm("{\n\t.reg .b8 t;\n\tcvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\tcvt.u32.u8 %0, t;\n\t}"
+        : "=r"(r)
+        : "f"(hi), "f"(lo));
     return r;
 }
 
@@ -259,6 +289,14 @@ __device__ __forceinline__ float div_by_const(float a, float c, float rc) {
     return __fmaf_rn(r, rc, q);
 }
 
+// The same for FMAX = 6 (E2M1): 6 = 1.5 * 2^2, so the byte is
+// E(amax) - 2 + [mantissa > 0x400000].  Checked exhaustively against the
+// division rule over every fp32 amax >= 1e-10.
+__device__ __forceinline__ uint32_t ue8m0_exponent_e2m1(float amax) {
+    const uint32_t b = __float_as_uint(amax);
+    return ((b >> 23) & 0xFFu) - 2u + ((b & 0x7FFFFFu) > 0x400000u ? 1u : 0u);
+}
+
 struct GroupScale {
     float mult;   // UE8M0: 2^(127-e) (exact); fp32 kinds: y = RN(1/s)
     float neg_s;  // fp32 kinds: -s
@@ -270,8 +308,8 @@ template <Kind KIND>
 __device__ __forceinline__ GroupScale make_scale(float amax) {
     GroupScale gs;
     amax = fmaxf(amax, 1e-10f);   // EPS floor
-    if constexpr (KIND == Kind::E4M3_UE8M0) {
-        gs.e8 = ue8m0_exponent(amax);
+    if constexpr (is_ue8m0(KIND)) {
+        gs.e8 = KIND == Kind::E2M1_UE8M0 ? ue8m0_exponent_e2m1(amax) : ue8m0_exponent(amax);
         gs.mult = __uint_as_float((254u - gs.e8) << 23);
         gs.s = 0.0f;
         gs.neg_s = 0.0f;
@@ -289,7 +327,20 @@ __device__ __forceinline__ GroupScale make_scale(float amax) {
 template <Kind KIND>
 __device__ __forceinline__ void encode16(const float (&v)[16], const GroupScale &gs,
                                          uint32_t (&w)[4]) {
-    if constexpr (KIND == Kind::E4M3_UE8M0) {
+    if constexpr (KIND == Kind::E2M1_UE8M0) {
+        // 16 codes in 8 bytes: w[0] elements 0..7, w[1] elements 8..15
+        const float2 m2 = make_float2(gs.mult, gs.mult);
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            uint32_t word = 0;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const float2 t = __fmul2_rn(make_float2(v[8 * j + 2 * k], v[8 * j + 2 * k + 1]), m2);
+                word |= e2m1x2(t.x, t.y) << (8 * k);
+            }
+            w[j] = word;
+        }
+    } else if constexpr (KIND == Kind::E4M3_UE8M0) {
         const float2 m2 = make_float2(gs.mult, gs.mult);
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
@@ -526,23 +577,34 @@ __device__ __forceinline__ void quantize_strip(const uint32_t (&x)[8], const uin
     uint32_t w[4];
     GroupScale gs;
 
-    constexpr bool kMixed = PQG_UE8M0_MIXED && KIND == Kind::E4M3_UE8M0 && !FUSED &&
+    constexpr bool kMixed = PQG_UE8M0_MIXED && is_ue8m0(KIND) && !FUSED &&
                             std::is_same<In, __nv_bfloat16>::value;
     if constexpr (kMixed) {
         // absmax on the raw bits, t = x * 2^k by a mixed bf16 FMA: no widening
         uint32_t ab = absmax_bits16(x);
 #pragma unroll
         for (int o = 1; o < L; o <<= 1) ab = max(ab, __shfl_xor_sync(0xFFFFFFFFu, ab, o));
-        gs.e8 = ue8m0_exponent(fmaxf(__uint_as_float(ab << 16), 1e-10f));
+        const float amax = fmaxf(__uint_as_float(ab << 16), 1e-10f);
+        gs.e8 = KIND == Kind::E2M1_UE8M0 ? ue8m0_exponent_e2m1(amax) : ue8m0_exponent(amax);
         const uint16_t p2 = static_cast<uint16_t>((254u - gs.e8) << 7);  // bf16 2^(127-e)
+        if constexpr (KIND == Kind::E2M1_UE8M0) {
+            w[0] = w[1] = 0u;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const uint32_t a = x[2 * j], b = x[2 * j + 1];
-            const float t0 = mul_bf16_pow2(static_cast<uint16_t>(a & 0xFFFFu), p2);
-            const float t1 = mul_bf16_pow2(static_cast<uint16_t>(a >> 16), p2);
-            const float t2 = mul_bf16_pow2(static_cast<uint16_t>(b & 0xFFFFu), p2);
-            const float t3 = mul_bf16_pow2(static_cast<uint16_t>(b >> 16), p2);
-            w[j] = e4m3x2(t0, t1) | (e4m3x2(t2, t3) << 16);
+            for (int i = 0; i < 8; ++i) {
+                const float t0 = mul_bf16_pow2(static_cast<uint16_t>(x[i] & 0xFFFFu), p2);
+                const float t1 = mul_bf16_pow2(static_cast<uint16_t>(x[i] >> 16), p2);
+                w[i >> 2] |= e2m1x2(t0, t1) << (8 * (i & 3));
+            }
+        } else {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const uint32_t a = x[2 * j], b = x[2 * j + 1];
+                const float t0 = mul_bf16_pow2(static_cast<uint16_t>(a & 0xFFFFu), p2);
+                const float t1 = mul_bf16_pow2(static_cast<uint16_t>(a >> 16), p2);
+                const float t2 = mul_bf16_pow2(static_cast<uint16_t>(b & 0xFFFFu), p2);
+                const float t3 = mul_bf16_pow2(static_cast<uint16_t>(b >> 16), p2);
+                w[j] = e4m3x2(t0, t1) | (e4m3x2(t2, t3) << 16);
+            }
         }
     } else {
         float v[16];
@@ -567,7 +629,7 @@ __device__ __forceinline__ void quantize_strip(const uint32_t (&x)[8], const uin
     }
 
     uint32_t packed_word = 0;
-    if constexpr (KIND == Kind::E4M3_UE8M0) {
+    if constexpr (is_ue8m0(KIND)) {
         // little-endian word of groups 4j..4j+3 assembled across the 4 groups'
         // lanes (invalid groups contribute 0)
         packed_word = ok ? (gs.e8 << (8u * (g & 3u))) : 0u;
@@ -576,8 +638,11 @@ __device__ __forceinline__ void quantize_strip(const uint32_t (&x)[8], const uin
     }
     if (!ok) return;
 
-    store16B(p.out + e * p.out_expert_bytes + static_cast<uint64_t>(row) * p.K + col, w[0], w[1],
-             w[2], w[3]);
+    uint8_t *dst = p.out + e * p.out_expert_bytes + static_cast<uint64_t>(row) * p.out_row_bytes;
+    if constexpr (KIND == Kind::E2M1_UE8M0)
+        store8B(dst + col / 2u, w[0], w[1]);
+    else
+        store16B(dst + col, w[0], w[1], w[2], w[3]);
     if (sub == 0) {
         uint8_t *sc = p.scales + e * p.scale_expert_bytes;
         if (p.layout == kPacked) {
@@ -589,7 +654,7 @@ __device__ __forceinline__ void quantize_strip(const uint32_t (&x)[8], const uin
         } else {
             const uint64_t idx = (p.layout == kRowMajor) ? static_cast<uint64_t>(row) * p.ng + g
                                                          : static_cast<uint64_t>(g) * p.mpad + row;
-            if constexpr (KIND == Kind::E4M3_UE8M0)
+            if constexpr (is_ue8m0(KIND))
                 sc[idx] = static_cast<uint8_t>(gs.e8);
             else
                 reinterpret_cast<float *>(sc)[idx] = gs.s;
@@ -620,7 +685,7 @@ __device__ __forceinline__ void quantize_chunk(const Chunk<ITEMS, FUSED> &ch, co
 #endif
 template <Kind KIND, bool FUSED>
 constexpr int min_blocks() {
-    return (KIND != Kind::E4M3_UE8M0 && !FUSED) ? PQG_MIN_BLOCKS_FP32 : 0;
+    return (!is_ue8m0(KIND) && !FUSED) ? PQG_MIN_BLOCKS_FP32 : 0;
 }
 
 template <typename In, int G, Kind KIND, bool FUSED, int ITEMS, int WARPS, bool MULTI>

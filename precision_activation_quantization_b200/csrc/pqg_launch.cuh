@@ -126,6 +126,7 @@ cudaError_t launch_group(const LaunchArgs &a) {
         case Kind::E4M3_FP32: return launch_kind<In, G, Kind::E4M3_FP32>(a);
         case Kind::E4M3_UE8M0: return launch_kind<In, G, Kind::E4M3_UE8M0>(a);
         case Kind::INT8_FP32: return launch_kind<In, G, Kind::INT8_FP32>(a);
+        case Kind::E2M1_UE8M0: return launch_kind<In, G, Kind::E2M1_UE8M0>(a);
     }
     return cudaErrorInvalidValue;
 }
@@ -134,15 +135,21 @@ cudaError_t launch_group(const LaunchArgs &a) {
 // Per-token (G = K) launches
 // ---------------------------------------------------------------------------
 
-// Warps sharing a row and 16-element slots per thread for a row of K outputs.
+// Warps sharing a row and 16-element slots per thread for a row of K outputs:
+// at most PQG_ROW_SLOTS slots per thread while 8 warps suffice, 4 beyond.
+#ifndef PQG_ROW_SLOTS
+#define PQG_ROW_SLOTS 2
+#endif
 inline void row_shape(uint32_t K, uint32_t *wpr, int *slots) {
     const uint32_t nslots = K / 16u;
-    if (nslots <= 32) { *wpr = 1; *slots = 1; }
-    else if (nslots <= 64) { *wpr = 1; *slots = 2; }
-    else if (nslots <= 128) { *wpr = 1; *slots = 4; }
-    else if (nslots <= 256) { *wpr = 2; *slots = 4; }
-    else if (nslots <= 512) { *wpr = 4; *slots = 4; }
-    else { *wpr = 8; *slots = 4; }
+    const uint32_t cap = PQG_ROW_SLOTS;
+    *slots = 1;
+    *wpr = 1;
+    while (*wpr * 32u * static_cast<uint32_t>(*slots) < nslots) {
+        if (static_cast<uint32_t>(*slots) < cap) *slots *= 2;
+        else if (*wpr < 8u) *wpr *= 2;
+        else *slots *= 2;  // K > 256 * 16 * cap: up to 4 slots
+    }
 }
 
 template <typename In, Kind KIND, bool FUSED, int SLOTS>
@@ -208,6 +215,8 @@ cudaError_t launch_row(const LaunchArgs &a) {
         case Kind::INT8_FP32:
             return a.fused ? launch_row_kind<In, Kind::INT8_FP32, true>(a)
                            : launch_row_kind<In, Kind::INT8_FP32, false>(a);
+        case Kind::E2M1_UE8M0:
+            break;  // rejected by the caller: MXFP4 groups are 32/64/128 wide
     }
     return cudaErrorInvalidValue;
 }

@@ -25,6 +25,7 @@ constexpr int kRowThreads = 256;  // 8 warps per CTA
 template <typename In, Kind KIND, bool FUSED, int SLOTS>
 __global__ void __launch_bounds__(kRowThreads)
     row_quant_kernel(const __grid_constant__ Params p) {
+    static_assert(KIND != Kind::E2M1_UE8M0, "per-token E2M1 is not offered");
     extern __shared__ __align__(16) uint32_t smem_prefix[];
     __shared__ float partial[2][kRowThreads / 32];
 
@@ -120,7 +121,7 @@ __global__ void __launch_bounds__(kRowThreads)
                     reinterpret_cast<uint32_t *>(sc)[row] = gs.e8;  // bytes 1..3 are 0
                 else if (p.layout == kTiled128x4)
                     store_tiled(sc, row, 0u, 1u, gs.e8);
-                else if constexpr (KIND == Kind::E4M3_UE8M0)
+                else if constexpr (is_ue8m0(KIND))
                     sc[row] = static_cast<uint8_t>(gs.e8);
                 else
                     reinterpret_cast<float *>(sc)[row] = gs.s;

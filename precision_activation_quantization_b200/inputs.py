@@ -108,8 +108,8 @@ class Workload:
         """
         ng = self.K // self.group
         in_row = (2 if self.fused else 1) * self.K * 2
-        out_row = self.K
-        if self.layout == "packed":
+        out_row = self.K // 2 if self.out_dtype == "e2m1" else self.K
+        if self.layout in ("packed", "tile128x4"):
             scale_row = 4 * ((ng + 3) // 4)
         else:
             scale_row = ng * (1 if self.scale_fmt == "ue8m0" else 4)
@@ -181,6 +181,13 @@ def masked(E: int = 32, M_max: int = 2048, K: int = 2048, seed: int = 4,
     name = f"masked{'_decode' if decode else ''}_{E}x{M_max}x2x{K}"
     return Workload(name, x, M=M_max, K=K, E=E, scale_fmt="ue8m0", layout="col",
                     fused=True, masked_m=mm, expected_m=expected)
+
+
+def mxfp4(M: int = 8192, K: int = 7168, seed: int = 1) -> Workload:
+    """The flat hidden-state input as an MXFP4 operand: G = 32, E2M1 codes, UE8M0
+    scales in the 128x4 tiled layout."""
+    w = flat_hidden(M=M, K=K, seed=seed)
+    return w.with_(name=f"mxfp4_{M}x{K}", group=32, out_dtype="e2m1", layout="tile128x4")
 
 
 def sweep(M: int, K: int = 4096, in_dtype: str = "bf16", group: int = 128,

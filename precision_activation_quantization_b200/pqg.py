@@ -27,12 +27,12 @@ PQG_ERR_UNSUPPORTED = -2
 PQG_ERR_ALIGNMENT = -3
 PQG_ERR_CUDA = -4
 
-PQG_BF16, PQG_FP16, PQG_E4M3, PQG_INT8 = 0, 1, 2, 3
+PQG_BF16, PQG_FP16, PQG_E4M3, PQG_INT8, PQG_E2M1 = 0, 1, 2, 3, 4
 PQG_SCALE_FP32, PQG_SCALE_UE8M0 = 0, 1
 PQG_ROW_MAJOR, PQG_COL_MAJOR_TMA, PQG_UE8M0_PACKED, PQG_UE8M0_TILED_128x4 = 0, 1, 2, 3
 
 IN_DTYPES = {"bf16": PQG_BF16, "fp16": PQG_FP16}
-OUT_DTYPES = {"e4m3": PQG_E4M3, "int8": PQG_INT8}
+OUT_DTYPES = {"e4m3": PQG_E4M3, "int8": PQG_INT8, "e2m1": PQG_E2M1}
 SCALE_FMTS = {"fp32": PQG_SCALE_FP32, "ue8m0": PQG_SCALE_UE8M0}
 LAYOUTS = {"row": PQG_ROW_MAJOR, "col": PQG_COL_MAJOR_TMA, "packed": PQG_UE8M0_PACKED,
            "tile128x4": PQG_UE8M0_TILED_128x4}
@@ -142,10 +142,14 @@ def scales_spec(M: int, K: int, group: int, scale_fmt: str = "fp32", layout: str
 def allocate_outputs(M: int, K: int, group: int, *, num_experts: int = 1,
                      out_dtype: str = "e4m3", scale_fmt: str = "fp32", layout: str = "row",
                      device=None):
-    """Allocate (out, scales) for one call with torch (device memory only)."""
+    """Allocate (out, scales) for one call with torch (device memory only).
+    E2M1 codes come back as uint8 [E, M, K/2], two codes per byte."""
     import torch
-    odt = torch.float8_e4m3fn if out_dtype == "e4m3" else torch.int8
-    out = torch.empty((num_experts, M, K), dtype=odt, device=device)
+    if out_dtype == "e2m1":
+        out = torch.empty((num_experts, M, K // 2), dtype=torch.uint8, device=device)
+    else:
+        odt = torch.float8_e4m3fn if out_dtype == "e4m3" else torch.int8
+        out = torch.empty((num_experts, M, K), dtype=odt, device=device)
     shape, sdt = scales_spec(M, K, group, scale_fmt, layout, num_experts)
     return out, torch.empty(shape, dtype=sdt, device=device)
 
@@ -197,11 +201,12 @@ def quant(x, out=None, scales=None, *, M: int | None = None, K: int | None = Non
                                 scale_fmt=scale_fmt, layout=layout, device=x.device)
         out = o if out is None else out
         scales = s if scales is None else scales
-    odt = torch.float8_e4m3fn if out_dtype == "e4m3" else torch.int8
+    odt = {"e4m3": torch.float8_e4m3fn, "int8": torch.int8, "e2m1": torch.uint8}[out_dtype]
+    out_bytes = E * M * (K // 2 if out_dtype == "e2m1" else K)
     if x.numel() != E * M * width:
         raise ValueError("x does not hold E x M rows of the given width")
-    if out.numel() * out.element_size() != E * M * K or out.dtype not in (odt, torch.uint8):
-        raise ValueError("out must hold E x M x K one-byte codes")
+    if out.numel() * out.element_size() != out_bytes or out.dtype not in (odt, torch.uint8):
+        raise ValueError(f"out must hold {out_bytes} bytes of codes")
     nbytes = pqg_scales_bytes(E, M, K, group, SCALE_FMTS[scale_fmt], LAYOUTS[layout])
     if nbytes >= 0 and scales.numel() * scales.element_size() != nbytes:
         raise ValueError(f"scales must be {nbytes} bytes for this layout")

@@ -25,7 +25,7 @@ def _torch_input(w):
 def run_gpu(w, *, expected_m=None, stream=None, x_dev=None):
     """Run ``w`` through pqg_quant; returns (codes uint8 [E*M*K], scale bytes)."""
     x = _torch_input(w) if x_dev is None else x_dev
-    n_out = w.E * w.M * w.K
+    n_out = w.E * w.M * (w.K // 2 if w.out_dtype == "e2m1" else w.K)
     nbytes = pqg.pqg_scales_bytes(w.E, w.M, w.K, w.group, pqg.SCALE_FMTS[w.scale_fmt],
                                   pqg.LAYOUTS[w.layout])
     assert nbytes >= 0
@@ -82,6 +82,14 @@ def _e4m3_values() -> np.ndarray:
 
 
 E4M3 = _e4m3_values()
+E2M1 = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0] + [-0.0, -0.5, -1.0, -1.5, -2.0, -3.0,
+                                                          -4.0, -6.0])
+E2M1_RANK = np.searchsorted(np.sort(np.unique(E2M1)), E2M1)   # code -> position, +-0 merged
+
+
+def _unpack_e2m1(b: np.ndarray) -> np.ndarray:
+    """[..., K/2] bytes -> [..., K] 4-bit codes (element 2i in the low nibble)."""
+    return np.stack([b & 0xF, b >> 4], axis=-1).reshape(*b.shape[:-1], -1)
 _FINITE = np.sort(np.unique(E4M3[~np.isnan(E4M3)]))     # -448 .. 448, one zero
 E4M3_RANK = np.searchsorted(_FINITE, np.nan_to_num(E4M3))  # code -> position
 
@@ -128,8 +136,11 @@ def check_fused(w, *, max_flip_frac=1e-4, rel_tol=7e-2, **kw):
     live = np.arange(M)[None, :] < rows[:, None]                       # [E, M]
 
     # untouched rows and padding must be byte-identical (sentinels)
-    gq3, rq3 = gq.reshape(E, M, K), rq.reshape(E, M, K)
+    kb = K // 2 if w.out_dtype == "e2m1" else K
+    gq3, rq3 = gq.reshape(E, M, kb), rq.reshape(E, M, kb)
     assert_same(gq3[~live], rq3[~live], f"{w.name} masked-off codes")
+    if w.out_dtype == "e2m1":
+        gq3, rq3 = _unpack_e2m1(gq3), _unpack_e2m1(rq3)
     g_sc, g_e8 = _scale_planes(w, gs)
     r_sc, r_e8 = _scale_planes(w, rs)
     # scale bytes outside live (row, group) cells must be untouched
@@ -187,6 +198,8 @@ def check_fused(w, *, max_flip_frac=1e-4, rel_tol=7e-2, **kw):
     n_el = gcodes.size
     if w.out_dtype == "int8":
         step = np.abs(gcodes.view(np.int8).astype(np.int64) - rcodes.view(np.int8).astype(np.int64))
+    elif w.out_dtype == "e2m1":
+        step = np.abs(E2M1_RANK[gcodes].astype(np.int64) - E2M1_RANK[rcodes].astype(np.int64))
     else:
         step = np.abs(E4M3_RANK[gcodes].astype(np.int64) - E4M3_RANK[rcodes].astype(np.int64))
     assert (step[diff] <= 1).all(), f"{w.name}: a code moved by more than one step"
@@ -195,13 +208,18 @@ def check_fused(w, *, max_flip_frac=1e-4, rel_tol=7e-2, **kw):
 
     # dequantized GPU value vs the oracle's y, per element
     vals = (gcodes.view(np.int8).astype(np.float64) if w.out_dtype == "int8"
-            else E4M3[gcodes])
+            else E2M1[gcodes] if w.out_dtype == "e2m1" else E4M3[gcodes])
     deq = vals * g_sc[..., None]
     yl = y[live].reshape(-1, K // G, G)
     t = np.abs(yl) / g_sc[..., None]
     err = np.abs(deq - yl)
     if w.out_dtype == "int8":
         assert (err <= (0.5 + 1.0) * g_sc[..., None]).all()
+    elif w.out_dtype == "e2m1":
+        # one step of E2M1 is at most half the value (normal) or 0.5 * s
+        big = t >= 1.0
+        assert (err[big] <= 0.5 * np.abs(yl[big]) + 1e-30).all(), f"{w.name}: dequant error"
+        assert (err[~big] <= np.broadcast_to(g_sc[..., None], t.shape)[~big] * 0.75).all()
     else:
         big = t >= 2.0 ** -6
         assert (err[big] <= rel_tol * np.abs(yl[big])).all(), f"{w.name}: dequant error"

@@ -78,7 +78,7 @@ def test_status_strings_and_version():
 def test_enum_values_match_header():
     text = open(HEADER).read()
     for name in ("PQG_OK", "PQG_ERR_INVALID_ARG", "PQG_ERR_UNSUPPORTED", "PQG_ERR_ALIGNMENT",
-                 "PQG_ERR_CUDA", "PQG_BF16", "PQG_FP16", "PQG_E4M3", "PQG_INT8",
+                 "PQG_ERR_CUDA", "PQG_BF16", "PQG_FP16", "PQG_E4M3", "PQG_INT8", "PQG_E2M1",
                  "PQG_SCALE_FP32", "PQG_SCALE_UE8M0", "PQG_ROW_MAJOR", "PQG_COL_MAJOR_TMA",
                  "PQG_UE8M0_PACKED", "PQG_UE8M0_TILED_128x4"):
         m = re.search(rf"\b{name}\s*=\s*(-?\d+)", text)
@@ -165,6 +165,9 @@ def call(**kw):
     (dict(out_dtype=pqg.PQG_INT8, scale_fmt=pqg.PQG_SCALE_UE8M0), pqg.PQG_ERR_UNSUPPORTED),
     (dict(scale_layout=pqg.PQG_UE8M0_PACKED), pqg.PQG_ERR_UNSUPPORTED),
     (dict(scale_layout=pqg.PQG_UE8M0_TILED_128x4), pqg.PQG_ERR_UNSUPPORTED),
+    (dict(out_dtype=pqg.PQG_E2M1), pqg.PQG_ERR_UNSUPPORTED),                 # needs UE8M0
+    (dict(out_dtype=pqg.PQG_E2M1, scale_fmt=pqg.PQG_SCALE_UE8M0, group=256), pqg.PQG_ERR_UNSUPPORTED),
+    (dict(out_dtype=5), pqg.PQG_ERR_INVALID_ARG),
     (dict(scale_layout=4), pqg.PQG_ERR_INVALID_ARG),
     (dict(in_ptr=0), pqg.PQG_ERR_INVALID_ARG),
     (dict(out_ptr=0), pqg.PQG_ERR_INVALID_ARG),

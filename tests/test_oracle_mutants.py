@@ -20,7 +20,8 @@ PINS = os.path.join(ROOT, "tests", "test_oracle_pins.py")
 
 MUTANTS = {
     "ue8m0_no_bump": ("int bump = (bits & 0x7FFFFF) != 0;", "int bump = 0;"),
-    "e4m3_ties_away": ("double n = nearbyint(a / quantum);", "double n = round(a / quantum);"),
+    "e4m3_ties_away": ("double n = nearbyint(a / quantum); /* exact quotient; ties to even */",
+                       "double n = round(a / quantum); /* exact quotient; ties to even */"),
     "e4m3_zero_sign_lost": ("uint8_t sign = signbit(t) ? 0x80 : 0x00;",
                             "uint8_t sign = (t < 0) ? 0x80 : 0x00;"),
     "e4m3_no_saturation": ("if (a > 448.0) a = 448.0;", ";"),
@@ -39,6 +40,10 @@ MUTANTS = {
     "packed_padding_not_zeroed": ("((uint8_t *)scales)[word * 4 + b] = 0;", ";"),
     "fp16_subnormal_exponent": ("v = ldexp((double)m, -24);", "v = ldexp((double)m, -25);"),
     "int8_truncates": ("double n = nearbyint((double)t);", "double n = trunc((double)t);"),
+    "e2m1_ties_away": ("double n = nearbyint(a / quantum);        /* ties to even */",
+                       "double n = round(a / quantum);        /* ties to even */"),
+    "mxfp4_uses_fmax448": ("ebyte = pqgo_ue8m0_exponent_fmax(amax, out_e2m1 ? PQGO_FMAX_E2M1",
+                           "ebyte = pqgo_ue8m0_exponent_fmax(amax, out_e2m1 ? PQGO_FMAX_E4M3"),
     "tile_rows_not_interleaved": ("(r % 32) * 16 + (r / 32) * 4", "(r % 32) * 4 + (r / 32) * 128"),
 }
 

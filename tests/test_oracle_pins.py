@@ -161,6 +161,65 @@ def test_e4m3_encoder_matches_torch_cast():
     assert np.array_equal(oracle.e4m3_encode(t), ref.view(torch.uint8).numpy())
 
 
+E2M1_MAGS = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+
+
+def brute_e2m1(t) -> np.ndarray:
+    """Nearest OCP E2M1 magnitude by exhaustive search (ties to the even code),
+    |t| clamped to 6, sign bit from t."""
+    t = np.asarray(t, np.float64).reshape(-1)
+    a = np.minimum(np.abs(t), 6.0)
+    d = np.abs(a[:, None] - E2M1_MAGS[None, :])
+    is_min = d == d.min(axis=1, keepdims=True)
+    codes = np.arange(8)
+    pick = np.where((is_min.sum(1) == 1)[:, None], is_min, is_min & (codes % 2 == 0)[None, :])
+    assert (pick.sum(1) == 1).all()
+    return (codes[pick.argmax(1)] | (np.signbit(t).astype(np.int64) << 3)).astype(np.uint8)
+
+
+def test_e2m1_encoder_matches_brute_force():
+    rng = np.random.default_rng(17)
+    _, bf = all_bf16_finite()
+    bf = bf[np.abs(bf) <= 16.0]
+    mids = (E2M1_MAGS[1:] + E2M1_MAGS[:-1]) / 2
+    mids = np.concatenate([mids, np.nextafter(mids.astype(np.float32), np.float32(9)),
+                           np.nextafter(mids.astype(np.float32), np.float32(-9))])
+    t = np.concatenate([bf, mids, -mids, rng.uniform(-8, 8, 100_000),
+                        np.float32([0.0, -0.0, 6.0, -6.0, 6.5, 1e9])]).astype(np.float32)
+    assert np.array_equal(oracle.e2m1_encode(t), brute_e2m1(t))
+
+
+def test_ue8m0_with_fmax6_equals_exact_ceiling():
+    rng = np.random.default_rng(18)
+    _, bf = all_bf16_finite()
+    a = np.concatenate([bf[bf >= 1e-10],
+                        rng.integers(np.float32(1e-10).view(np.uint32),
+                                     np.float32(2.0 ** 120).view(np.uint32), 1_000_000,
+                                     dtype=np.uint32).view(np.float32)]).astype(np.float32)
+    a64 = a.astype(np.float64)
+    n = np.floor(np.log2(a64 / 6.0)).astype(np.int64) - 2
+    for _ in range(6):
+        n = np.where(6.0 * np.exp2(n.astype(np.float64)) >= a64, n, n + 1)
+    for _ in range(6):
+        n = np.where(6.0 * np.exp2((n - 1).astype(np.float64)) >= a64, n - 1, n)
+    assert np.array_equal(oracle.ue8m0_exponent_fmax(a, 6.0).astype(np.int64), n + 127)
+
+
+def test_mxfp4_dequant_error_bound_and_nibble_order():
+    w = inputs.sweep(M=128, K=1024)
+    q, s = oracle.quant(w.x, M=w.M, K=w.K, group=32, out_dtype="e2m1", scale_fmt="ue8m0")
+    x = _f32(w.x).reshape(w.M, -1, 32).astype(np.float64)
+    lo, hi = q.reshape(w.M, -1) & 0xF, q.reshape(w.M, -1) >> 4
+    codes = np.stack([lo, hi], axis=-1).reshape(w.M, -1, 32)      # element 2i low nibble
+    vals = E2M1_MAGS[codes & 7] * np.where(codes & 8, -1.0, 1.0)
+    sc = np.exp2(s.reshape(w.M, -1, 1).astype(np.float64) - 127)
+    err = np.abs(vals * sc - x)
+    t = np.abs(x) / sc
+    assert (t <= 6.0).all()
+    assert (err[t >= 1] <= 0.25 * np.abs(x[t >= 1]) * (1 + 2.0 ** -20)).all()
+    assert (err[t < 1] <= 0.25 * np.broadcast_to(sc, x.shape)[t < 1] + 1e-30).all()
+
+
 def test_int8_encoder_matches_numpy_rint():
     rng = np.random.default_rng(13)
     t = np.concatenate([rng.uniform(-200, 200, 500_000).astype(np.float32),
@@ -224,6 +283,16 @@ def _golden_group(entry) -> np.ndarray:
 
 @pytest.mark.parametrize("entry", json.load(open(GOLDEN))["groups"], ids=lambda e: e["name"])
 def test_worked_group(entry):
+    if "e2m1" in entry:
+        v = np.zeros(entry["group"], np.float32)
+        for i, x in entry["values"].items():
+            v[int(i)] = x
+        q, s = oracle.quant(inputs.bf16_bits(v), M=1, K=entry["group"], group=entry["group"],
+                            out_dtype="e2m1", scale_fmt="ue8m0", layout="row")
+        assert int(s.reshape(-1)[0]) == entry["e2m1"]["exponent"]
+        for i, b in entry["e2m1"]["bytes"].items():
+            assert int(q.reshape(-1)[int(i)]) == b, (entry["name"], i)
+        return
     v = _golden_group(entry)
     bits = inputs.bf16_bits(v)
     assert np.array_equal(oracle.decode(bits).view(np.uint32), v.view(np.uint32)), \

@@ -338,3 +338,50 @@ def test_varlen_contiguous_equals_masked(kind):
         assert_same(fq[off[e]:off[e] + n].reshape(-1), mq[e, :n].reshape(-1), f"codes e={e}")
         assert_same(fs[off[e]:off[e] + n].view(np.uint8).reshape(-1),
                     ms[e, :n].view(np.uint8).reshape(-1), f"scales e={e}")
+
+
+# --------------------------------------------------------------------------
+# MXFP4: E2M1 codes (two per byte) with UE8M0 scales
+# --------------------------------------------------------------------------
+
+MX_LAYOUTS = ["row", "col", "packed", "tile128x4"]
+
+
+@pytest.mark.parametrize("layout", MX_LAYOUTS)
+@pytest.mark.parametrize("G", [32, 64, 128])
+@pytest.mark.parametrize("in_dtype", ["bf16", "fp16"])
+def test_mxfp4_bit_exact(layout, G, in_dtype):
+    for M, K in [(37, 640), (5, 128), (130, 2048), (1, 7168)]:
+        check_exact(make(M, K, G, ("e2m1", "ue8m0", layout), in_dtype, seed=M + K + G + 7))
+
+
+@pytest.mark.parametrize("layout", ["row", "tile128x4"])
+def test_mxfp4_fused_and_masked(layout):
+    E, M, K = 5, 37, 640
+    mm = np.array([0, 37, 1, 99, -3], np.int32)
+    check_exact(make(M, K, 32, ("e2m1", "ue8m0", layout), E=E, seed=51, masked_m=mm,
+                     expected_m=8))
+    check_fused(make(M, K, 32, ("e2m1", "ue8m0", layout), fused=True, E=E, seed=52,
+                     masked_m=mm, expected_m=8), max_flip_frac=1e-3)
+    check_fused(make(130, 2048, 32, ("e2m1", "ue8m0", layout), fused=True, seed=53),
+                max_flip_frac=1e-3)
+
+
+@pytest.mark.parametrize("in_dtype", ["bf16", "fp16"])
+@pytest.mark.parametrize("carrier", [6.0, 1.0, 1000.0])
+def test_mxfp4_every_input_value(in_dtype, carrier):
+    bits = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    import oracle
+    vals = oracle.decode(bits, in_dtype)
+    bits = bits[np.isfinite(vals)]
+    n = bits.size
+    cb = inputs.to_bits(np.float32([carrier]), in_dtype)[0]
+    x = np.full((1, n, 32), cb, np.uint16)
+    x[0, :, 0] = bits
+    x[0, :, 17] = bits ^ 0x8000
+    check_exact(inputs.Workload("exhaustive_e2m1", x, M=n, K=32, group=32, in_dtype=in_dtype,
+                                out_dtype="e2m1", scale_fmt="ue8m0", layout="row"))
+
+
+def test_mxfp4_full_size():
+    check_exact(inputs.mxfp4())

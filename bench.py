@@ -52,6 +52,7 @@ def workloads():
         "per_token": lambda: inputs.flat_hidden(layout="row", scale_fmt="fp32").with_(
             group=7168, name="per_token_8192x7168"),
         "mxfp4": lambda: inputs.mxfp4(),
+        "nvfp4": lambda: inputs.nvfp4(),
         "fused": lambda: inputs.fused(),
         "masked": lambda: inputs.masked(),
         "masked_decode": lambda: inputs.masked(decode=True),
@@ -66,20 +67,61 @@ def describe(w) -> dict:
         [w.M, 2 * w.K if w.fused else w.K]
     d = {"workload": w.name, "input_shape": shape, "in_dtype": w.in_dtype,
          "out_dtype": w.out_dtype, "group": w.group,
-         "scales": f"{w.scale_fmt} {dict(row='row-major', col='column-major TMA-aligned', packed='UE8M0-packed column-major', tile128x4='128x4 tiled (MX)')[w.layout]}",
+         "scales": f"{w.scale_fmt} {dict(row='row-major', col='column-major TMA-aligned', packed='UE8M0-packed column-major', tile128x4='128x4 tiled')[w.layout]}",
          "fused_silu_mul": w.fused, "rows_quantized": w.rows,
          "algorithmic_bytes_per_step": w.algorithmic_bytes()}
     if w.masked_m is not None:
         d["masked"] = {"experts": w.E, "M_max": w.M, "sum_masked_m": w.rows,
                        "expected_m": w.expected_m}
+    if w.global_scale is not None:
+        d["global_scale"] = w.global_scale
     return d
 
 
-def source_digest() -> str:
-    """sha256 over the CUDA sources, to tell whether stored ncu counters still apply."""
+def make_call(w, dev, M=None):
+    """The C entry point for ``w`` with every argument but the buffers bound:
+    call(in_ptr, out_ptr, scales_ptr, stream_handle) -> status.  NVFP4 goes
+    through pqg_quant_nvfp4 with its global scale in device memory."""
+    import torch
+    from precision_activation_quantization_b200 import pqg
+    M = w.M if M is None else M
+    E = w.E if M == w.M else 1
+    mm = None if (w.masked_m is None or E == 1 and M != w.M) else \
+        torch.from_numpy(w.masked_m).to(dev)
+    mm_ptr = None if mm is None else mm.data_ptr()
+    em = w.expected_m if mm is not None else 0
+    if w.scale_fmt == "e4m3":
+        gsc = torch.tensor([w.global_scale], dtype=torch.float32, device=dev)
+
+        def call(a, b, c, sh):
+            return pqg.pqg_quant_nvfp4(a, b, c, gsc.data_ptr(), M, E, w.K,
+                                       pqg.IN_DTYPES[w.in_dtype], pqg.LAYOUTS[w.layout],
+                                       int(w.fused), mm_ptr, em, sh)
+        call.keep = (gsc, mm)
+        return call
+
+    def call(a, b, c, sh):
+        return pqg.pqg_quant(a, b, c, M, E, w.K, w.group, pqg.IN_DTYPES[w.in_dtype],
+                             pqg.OUT_DTYPES[w.out_dtype], pqg.SCALE_FMTS[w.scale_fmt],
+                             pqg.LAYOUTS[w.layout], int(w.fused), mm_ptr, em, sh)
+    call.keep = (mm,)
+    return call
+
+
+def kernel_of(w) -> str:
+    """Which kernel a workload runs: "row" (per-token, G = K) or "strip"."""
+    return "row" if w.group == w.K and w.group not in (16, 32, 64, 128) else "strip"
+
+
+def source_digest(kernel: str = "strip") -> str:
+    """sha256 over the CUDA sources a kernel is built from (the strip kernel does
+    not include the per-token row kernel's file), to tell whether stored ncu
+    counters still apply."""
     csrc = os.path.join(ROOT, "precision_activation_quantization_b200", "csrc")
     h = hashlib.sha256()
     for f in sorted(os.listdir(csrc)):
+        if kernel == "strip" and f == "pqg_row_kernel.cuh":
+            continue
         with open(os.path.join(csrc, f), "rb") as fh:
             h.update(f.encode() + fh.read())
     return h.hexdigest()
@@ -93,11 +135,11 @@ def hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def stored_traffic(name: str):
+def stored_traffic(name: str, kernel: str = "strip"):
     try:
         with open(TRAFFIC_FILE) as f:
             rec = json.load(f).get(name)
-        if rec and rec.get("source_sha256") == source_digest():
+        if rec and rec.get("source_sha256") == source_digest(kernel):
             return rec["dram_bytes_per_launch"]
     except Exception:
         pass
@@ -201,7 +243,7 @@ def run_reference(args, w) -> dict:
         sub = w.with_(x=w.x[e:e + 1, m0:m0 + n], M=n, E=1, masked_m=None)
         oracle.quant(sub.x, M=n, K=w.K, group=w.group, in_dtype=w.in_dtype,
                      out_dtype=w.out_dtype, scale_fmt=w.scale_fmt, layout=w.layout,
-                     fused=w.fused)
+                     fused=w.fused, global_scale=w.global_scale)
         return sub.algorithmic_bytes(), n
 
     for i in range(args.warmup):
@@ -235,7 +277,7 @@ def cpu_baseline(w, budget_s: float = 10.0) -> dict:
     while True:
         oracle.quant(w.x, E=w.E, M=w.M, K=w.K, group=w.group, in_dtype=w.in_dtype,
                      out_dtype=w.out_dtype, scale_fmt=w.scale_fmt, layout=w.layout,
-                     fused=w.fused, masked_m=w.masked_m)
+                     fused=w.fused, masked_m=w.masked_m, global_scale=w.global_scale)
         reps += 1
         dt = time.perf_counter() - t0
         if dt >= budget_s or reps >= 50:
@@ -269,15 +311,12 @@ def run_ours(args, w, rank: int, world: int, local_rank: int) -> dict | None:
     xs = [x0] + [x0.clone() for _ in range(sets - 1)]
     outs = [torch.empty(n_out, dtype=torch.uint8, device=dev) for _ in range(sets)]
     scs = [torch.empty(max(nbytes, 1), dtype=torch.uint8, device=dev) for _ in range(sets)]
-    mm = None if w.masked_m is None else torch.from_numpy(w.masked_m).to(dev)
-    mm_ptr = None if mm is None else mm.data_ptr()
-    args_c = (w.M, w.E, w.K, w.group, pqg.IN_DTYPES[w.in_dtype], pqg.OUT_DTYPES[w.out_dtype],
-              pqg.SCALE_FMTS[w.scale_fmt], pqg.LAYOUTS[w.layout], int(w.fused))
+    call = make_call(w, dev)
     ptrs = [(xs[i].data_ptr(), outs[i].data_ptr(), scs[i].data_ptr()) for i in range(sets)]
 
     def launch(i):
         a, b, c = ptrs[i % sets]
-        st = pqg.pqg_quant(a, b, c, *args_c, mm_ptr, w.expected_m, sh)
+        st = call(a, b, c, sh)
         if st != pqg.PQG_OK:
             raise pqg.PqgError(st)
 
@@ -328,7 +367,7 @@ def run_ours(args, w, rank: int, world: int, local_rank: int) -> dict | None:
         # latency at M = 1 (same configuration, one row)
         lat = latency_m1(w, dev, stream) if rank == 0 else None
         # end to end: pinned host input -> device -> quantize -> codes/scales back
-        e2e = end_to_end(args, w, dev, stream, x0, outs[0], scs[0], mm_ptr, args_c, world)
+        e2e = end_to_end(args, w, dev, stream, x0, outs[0], scs[0], call, world)
 
     del xs, outs, scs
     torch.cuda.empty_cache()
@@ -337,7 +376,7 @@ def run_ours(args, w, rank: int, world: int, local_rank: int) -> dict | None:
 
     peak, peak_src = hbm_peak()
     achieved = bytes_step / (ms_step * 1e-3) / 1e9
-    traffic = stored_traffic(w.name)
+    traffic = stored_traffic(w.name, kernel_of(w))
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
@@ -355,7 +394,8 @@ def run_ours(args, w, rank: int, world: int, local_rank: int) -> dict | None:
                      "frac": achieved / peak, "peak_source": peak_src,
                      "traffic": traffic,
                      "algorithmic_bytes_per_launch": bytes_step,
-                     "kernel": "pqg::quant_kernel (one launch per step)"},
+                     "kernel": ("pqg::row_quant_kernel" if kernel_of(w) == "row"
+                                else "pqg::quant_kernel") + " (one launch per step)"},
         "e2e": e2e,
         "gpu_launches": launches,
         "clocks": clocks.summary(),
@@ -377,18 +417,17 @@ def latency_m1(w, dev, stream) -> dict:
     nb = pqg.pqg_scales_bytes(1, 1, w.K, w.group, pqg.SCALE_FMTS[w.scale_fmt],
                               pqg.LAYOUTS[w.layout])
     sc = torch.empty(nb, dtype=torch.uint8, device=dev)
-    a = (x.data_ptr(), out.data_ptr(), sc.data_ptr(), 1, 1, w.K, w.group,
-         pqg.IN_DTYPES[w.in_dtype], pqg.OUT_DTYPES[w.out_dtype], pqg.SCALE_FMTS[w.scale_fmt],
-         pqg.LAYOUTS[w.layout], int(w.fused), None, 0)
+    call = make_call(w, dev, M=1)
+    a = (x.data_ptr(), out.data_ptr(), sc.data_ptr())
     s = torch.cuda.Stream(dev)
     with torch.cuda.stream(s):
         for _ in range(10):
-            pqg.pqg_quant(*a, s.cuda_stream)
+            call(*a, s.cuda_stream)
         n = 200
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=s):
             for _ in range(n):
-                pqg.pqg_quant(*a, s.cuda_stream)
+                call(*a, s.cuda_stream)
         g.replay()
         torch.cuda.synchronize(dev)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -401,7 +440,7 @@ def latency_m1(w, dev, stream) -> dict:
         graph_us = e0.elapsed_time(e1) * 1e3 / (reps * n)
         e0.record(s)
         for _ in range(n):
-            pqg.pqg_quant(*a, s.cuda_stream)
+            call(*a, s.cuda_stream)
         e1.record(s)
         e1.synchronize()
         stream_us = e0.elapsed_time(e1) * 1e3 / n
@@ -411,7 +450,7 @@ def latency_m1(w, dev, stream) -> dict:
                     "(device time per call); stream = 200 back-to-back launches from Python"}
 
 
-def end_to_end(args, w, dev, stream, x_dev, out_dev, sc_dev, mm_ptr, args_c, world) -> dict:
+def end_to_end(args, w, dev, stream, x_dev, out_dev, sc_dev, call, world) -> dict:
     """Same metric through the public API with host buffers: every step copies its
     input from pinned host memory, quantizes, and reads codes and scales back."""
     import torch
@@ -426,8 +465,7 @@ def end_to_end(args, w, dev, stream, x_dev, out_dev, sc_dev, mm_ptr, args_c, wor
 
     def step():
         x_dev.copy_(x_host, non_blocking=True)
-        st = pqg.pqg_quant(x_dev.data_ptr(), out_dev.data_ptr(), sc_dev.data_ptr(), *args_c,
-                           mm_ptr, w.expected_m, sh)
+        st = call(x_dev.data_ptr(), out_dev.data_ptr(), sc_dev.data_ptr(), sh)
         if st != pqg.PQG_OK:
             raise pqg.PqgError(st)
         out_host.copy_(out_dev, non_blocking=True)

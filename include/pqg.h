@@ -88,7 +88,9 @@ enum pqg_dtype {
 /* Scale formats. */
 enum pqg_scale_fmt {
     PQG_SCALE_FP32 = 0,  /* one float per group                        */
-    PQG_SCALE_UE8M0 = 1  /* one biased exponent byte e, scale 2^(e-127) */
+    PQG_SCALE_UE8M0 = 1, /* one biased exponent byte e, scale 2^(e-127) */
+    PQG_SCALE_E4M3 = 2   /* one OCP E4M3 byte per block of 16 (NVFP4,
+                            pqg_quant_nvfp4 only)                       */
 };
 
 /* Scale layouts, per expert.  ng = K / group; M_pad = M rounded up to a
@@ -110,8 +112,9 @@ enum pqg_scale_fmt {
  *                       (row m, group g) is byte (m%32)*16 + ((m/32)%4)*4 + g%4.
  *                       Plane: ceil(M/128)*128 x ceil(ng/4)*4 bytes.  Bytes of
  *                       padding groups (>= ng) in a quantized row are written 0;
- *                       padding rows are not written.  UE8M0 only; with G = 32
- *                       this is the MXFP8 operand format.
+ *                       padding rows are not written.  UE8M0 bytes (with G = 32
+ *                       the MXFP8 operand format) or, through pqg_quant_nvfp4,
+ *                       E4M3 block-scale bytes (the NVFP4 operand format).
  * Expert e's plane starts pqg_scales_bytes(1, M, K, ...) * e bytes into the
  * buffer. */
 enum pqg_scale_layout {
@@ -146,7 +149,8 @@ enum pqg_scale_layout {
  *          is 2^ceil(log2(amax / 6)) by the same bit rule with FMAX = 6.
  * scale_fmt, scale_layout   see above.  PQG_SCALE_UE8M0 rejects PQG_INT8, and
  *          PQG_UE8M0_PACKED and PQG_UE8M0_TILED_128x4 require PQG_SCALE_UE8M0
- *          (else PQG_ERR_UNSUPPORTED).
+ *          (else PQG_ERR_UNSUPPORTED).  PQG_SCALE_E4M3 needs a global scale:
+ *          pqg_quant returns PQG_ERR_UNSUPPORTED for it (see pqg_quant_nvfp4).
  * fuse_silu_mul  nonzero: quantize silu(gate) * up (see the numerics above).
  * masked_m device, int32[num_experts], or NULL.  Masked dispatch (grouped-masked
  *          MoE): expert e quantizes only rows m < clamp(masked_m[e], 0, M); the
@@ -170,9 +174,47 @@ PQG_API int pqg_quant(const void *in, void *out, void *scales, int64_t M,
               const int32_t *masked_m, int64_t expected_m, pqg_stream_t stream);
 
 /*
- * pqg_scales_bytes — size in bytes of the scale buffer pqg_quant writes for
- * these arguments (all experts, padding rows included).  Returns a negative
- * pqg_status for arguments pqg_quant would reject.
+ * pqg_quant_nvfp4 — NVFP4 quantization ("block_size = 16 -> NVFP4", FlashInfer
+ * GEMM notes, section 6): E2M1 codes in blocks of 16 with an E4M3 block scale
+ * under a per-call fp32 global scale g.  The pages give only the block size;
+ * the arithmetic below is this library's reading of the two-level NVFP4 scale.
+ * Per block, in fp32 with round-to-nearest-even:
+ *   amax = max(max_i |x_i|, 1e-10f)
+ *   r    = (amax / 6) * g           two roundings, in this order
+ *   sf   = nearest E4M3 code of r, saturating at 448       (the stored byte)
+ *   mult = g / value(sf), or 0 when value(sf) == 0
+ *   code = nearest E2M1 value of x_i * mult, saturating at +-6 (zero keeps
+ *          the sign of the product)
+ * so x_i is approximately code * value(sf) / g.  Bit-identical to that
+ * definition for every non-fused call; the fused prologue follows pqg_quant's
+ * note.
+ *
+ * in, M, num_experts, in_dtype, fuse_silu_mul, masked_m, expected_m, stream:
+ *          as for pqg_quant.
+ * out      device.  [num_experts][M][K/2] bytes, two E2M1 codes per byte,
+ *          element 2i in bits 0-3.  16-byte aligned.
+ * scales   device.  pqg_scales_bytes(num_experts, M, K, 16, PQG_SCALE_E4M3,
+ *          scale_layout) bytes: one E4M3 byte per block in PQG_ROW_MAJOR,
+ *          PQG_COL_MAJOR_TMA or PQG_UE8M0_TILED_128x4 (the 128x4 tile holds
+ *          E4M3 bytes here); PQG_UE8M0_PACKED is rejected (PQG_ERR_UNSUPPORTED).
+ * global_scale  device, one fp32 g, finite and > 0 (else the codes are
+ *          unspecified; nothing faults).  Read on the device after the
+ *          programmatic-dependent-launch wait, so the preceding kernel on
+ *          `stream` may produce it (typically 448 * 6 / amax of the tensor).
+ *          4-byte aligned.
+ * K        a positive multiple of 16.
+ * Same limits and return codes as pqg_quant.
+ */
+PQG_API int pqg_quant_nvfp4(const void *in, void *out, void *scales,
+              const float *global_scale, int64_t M, int64_t num_experts, int64_t K,
+              int in_dtype, int scale_layout, int fuse_silu_mul,
+              const int32_t *masked_m, int64_t expected_m, pqg_stream_t stream);
+
+/*
+ * pqg_scales_bytes — size in bytes of the scale buffer pqg_quant (or, for
+ * PQG_SCALE_E4M3 with group 16, pqg_quant_nvfp4) writes for these arguments
+ * (all experts, padding rows included).  Returns a negative pqg_status for
+ * arguments the call would reject.
  */
 PQG_API int64_t pqg_scales_bytes(int64_t num_experts, int64_t M, int64_t K, int group,
                          int scale_fmt, int scale_layout);
@@ -188,7 +230,8 @@ PQG_API int pqg_last_cuda_error(void);
  * later pqg_quant calls of this process.  Returns the previous setting. */
 PQG_API int pqg_set_pdl(int enable);
 
-/* Number of kernels this process has launched through pqg_quant so far. */
+/* Number of kernels this process has launched through pqg_quant and
+ * pqg_quant_nvfp4 so far. */
 PQG_API uint64_t pqg_launch_count(void);
 
 /* Library version string, e.g. "pqg 0.1.0 sm_100a". */

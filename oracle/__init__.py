@@ -13,7 +13,7 @@ Source: sglang PR #30924 report, "[JIT] Trait-driven per_token_group_quant"
 (实现拆解 items 1-2; 关键源码片段 ``ref_fp8_ue8m0``; 风险与影响 on the INT8
 path), the TeleFuser "tf-kernel 安装与使用" page (使用示例, silu_and_mul halves)
 and "FlashInfer GEMM 学习笔记" §6-7 (packed TMA-aligned scales, masked_m /
-expected_m).
+expected_m, MXFP4 at block 32 and NVFP4 at block 16).
 """
 from __future__ import annotations
 
@@ -96,6 +96,13 @@ def load(path: str | None = None):
         lib.pqgo_ue8m0_exponent_fmax_n.argtypes = [vp, vp, i64, f32]
         lib.pqgo_scale_fp32_n.restype = None
         lib.pqgo_scale_fp32_n.argtypes = [vp, vp, i64, i32]
+        lib.pqgo_quant_nvfp4.restype = i32
+        lib.pqgo_quant_nvfp4.argtypes = [vp, vp, vp, i64, i64, i64, i32, i32, i32, vp, f32]
+        for name in ("pqgo_e4m3_decode_n", "pqgo_nvfp4_block_scale_n", "pqgo_nvfp4_multiplier_n"):
+            getattr(lib, name).restype = None
+        lib.pqgo_e4m3_decode_n.argtypes = [vp, vp, i64]
+        lib.pqgo_nvfp4_block_scale_n.argtypes = [vp, vp, i64, f32]
+        lib.pqgo_nvfp4_multiplier_n.argtypes = [vp, vp, i64, f32]
         if default:
             _lib = lib
         return lib
@@ -177,6 +184,32 @@ def scale_fp32(amax, out_dtype: str = "e4m3", lib=None) -> np.ndarray:
     return s
 
 
+def e4m3_decode(codes, lib=None) -> np.ndarray:
+    lib = lib or load()
+    c = _c(codes, np.uint8)
+    v = np.empty(c.shape, np.float32)
+    lib.pqgo_e4m3_decode_n(_ptr(c), _ptr(v), c.size)
+    return v
+
+
+def nvfp4_block_scale(amax, global_scale: float, lib=None) -> np.ndarray:
+    """E4M3 block-scale codes of blocks with these absmax values (NVFP4)."""
+    lib = lib or load()
+    a = _c(amax, np.float32)
+    sf = np.empty(a.shape, np.uint8)
+    lib.pqgo_nvfp4_block_scale_n(_ptr(a), _ptr(sf), a.size, float(global_scale))
+    return sf
+
+
+def nvfp4_multiplier(sf, global_scale: float, lib=None) -> np.ndarray:
+    """fp32 multipliers g / value(sf) (0 for a zero block scale)."""
+    lib = lib or load()
+    c = _c(sf, np.uint8)
+    m = np.empty(c.shape, np.float32)
+    lib.pqgo_nvfp4_multiplier_n(_ptr(c), _ptr(m), c.size, float(global_scale))
+    return m
+
+
 def group_amax(v, lib=None) -> float:
     lib = lib or load()
     v = _c(v, np.float32)
@@ -199,13 +232,13 @@ def scales_shape(E: int, M: int, K: int, group: int, scale_fmt: str, layout: str
         return (E, (M + 127) // 128 * ((ng + 3) // 4) * 512), np.uint8
     else:
         return (E, (ng + 3) // 4, mpad), np.int32
-    return shape, (np.uint8 if scale_fmt == "ue8m0" else np.float32)
+    return shape, (np.float32 if scale_fmt == "fp32" else np.uint8)
 
 
 def quant(x_bits, *, M: int, K: int, group: int, E: int = 1, in_dtype: str = "bf16",
           out_dtype: str = "e4m3", scale_fmt: str = "fp32", layout: str = "row",
           fused: bool = False, masked_m=None, out: np.ndarray | None = None,
-          scales: np.ndarray | None = None, fill: int = 0xA5, lib=None):
+          scales: np.ndarray | None = None, fill: int = 0xA5, global_scale=None, lib=None):
     """Run the oracle on host arrays.
 
     ``x_bits`` holds raw 16-bit patterns shaped [E, M, K] ([E, M, 2K] fused;
@@ -213,6 +246,8 @@ def quant(x_bits, *, M: int, K: int, group: int, E: int = 1, in_dtype: str = "bf
     prefilled (rows the call must not touch are then checked by the caller);
     otherwise they are allocated filled with ``fill``.  Returns (out, scales)
     shaped [E, M, K] ([E, M, K/2] for E2M1) and per ``scales_shape``.
+    NVFP4 is ``out_dtype="e2m1", scale_fmt="e4m3", group=16`` with the fp32
+    ``global_scale``.
     """
     lib = lib or load()
     x = _c(x_bits, np.uint16)
@@ -226,7 +261,7 @@ def quant(x_bits, *, M: int, K: int, group: int, E: int = 1, in_dtype: str = "bf
     if scales is None:
         scales = np.empty(shape, sdt)
         scales.view(np.uint8).fill(fill)
-    nbytes = lib.pqgo_scales_nbytes(E, M, K, group, int(scale_fmt == "ue8m0"),
+    nbytes = lib.pqgo_scales_nbytes(E, M, K, group, int(scale_fmt != "fp32"),
                                     LAYOUTS[layout])
     if scales.nbytes != nbytes or out.size != E * M * kbytes:
         raise ValueError("output buffers have the wrong size")
@@ -235,6 +270,15 @@ def quant(x_bits, *, M: int, K: int, group: int, E: int = 1, in_dtype: str = "bf
         mm = _c(masked_m, np.int32)
         if mm.size != E:
             raise ValueError("masked_m needs one entry per expert")
+    if scale_fmt == "e4m3":
+        if out_dtype != "e2m1" or group != 16 or global_scale is None:
+            raise ValueError("E4M3 block scales are NVFP4: e2m1 codes, group 16, a global scale")
+        rc = lib.pqgo_quant_nvfp4(_ptr(x), _ptr(out), _ptr(scales), E, M, K,
+                                  int(in_dtype == "fp16"), LAYOUTS[layout], int(bool(fused)),
+                                  None if mm is None else _ptr(mm), float(global_scale))
+        if rc != 0:
+            raise ValueError(f"oracle rejected the call (status {rc})")
+        return out, scales
     rc = lib.pqgo_quant(_ptr(x), _ptr(out), _ptr(scales), E, M, K, group,
                         int(in_dtype == "fp16"), OUT_KINDS[out_dtype],
                         int(scale_fmt == "ue8m0"), LAYOUTS[layout], int(bool(fused)),

@@ -39,6 +39,13 @@
  *   - FP4 (MXFP4, the FlashInfer notes' "block_size = 32 -> MXFP4"): OCP E2M1
  *     codes (largest magnitude 6), UE8M0 scales by the same rule with FMAX = 6,
  *     two codes per byte with element 2i in bits 0-3 and 2i+1 in bits 4-7.
+ *   - NVFP4 (the FlashInfer notes' "block_size = 16 -> NVFP4", section 6):
+ *     E2M1 codes in blocks of 16 with an E4M3 block scale and one fp32
+ *     global scale g per call (the encode-side factor, typically
+ *     448 * 6 / amax of the tensor).  Per block, in this order and in fp32:
+ *     r = (amax / 6) * g; sf = E4M3(r) (nearest, saturating at 448);
+ *     d = value of sf; m = g / d (0 when d is 0); t_i = x_i * m; codes =
+ *     E2M1(t_i), saturating at 6.  The dequantized value is code * d / g.
  *   - column-major layouts pad the row count to a multiple of 4 (16 bytes of
  *     fp32 or one int32 word per 4 rows), padding rows are never written.
  *   - the UE8M0-packed layout stores the exponents of groups 4j..4j+3 of a
@@ -67,6 +74,7 @@
 #define PQGO_FMAX_INT8 127.0f   /* INT8 scale divisor ([PR] ref_int8)          */
 #define PQGO_FMAX_E2M1 6.0f     /* largest finite OCP E2M1 value (MXFP4)       */
 #define PQGO_EPS 1e-10f         /* absmax floor ([PR] "不低于 EPS")             */
+#define PQGO_NVFP4_BLOCK 16     /* NVFP4 block size ([FI] section 6)           */
 
 /* output kinds and layouts understood by the oracle (numbered for the Python
  * wrapper) */
@@ -182,6 +190,16 @@ uint8_t pqgo_e4m3_encode(float t) {
     }
 }
 
+/* Value of an OCP E4M3 ("fn") code: (1 + m/8) * 2^(e - 7) for exponent
+ * field e >= 1, (m/8) * 2^-6 for e = 0; S.1111.111 is NaN. */
+float pqgo_e4m3_decode(uint8_t c) {
+    int e = (c >> 3) & 0xF, m = c & 0x7;
+    double v;
+    if (e == 15 && m == 7) return NAN;
+    v = (e == 0) ? ldexp((double)m / 8.0, -6) : ldexp(1.0 + (double)m / 8.0, e - 7);
+    return (float)((c & 0x80) ? -v : v);
+}
+
 /* Saturating cast to INT8: round to nearest integer, ties to even, then
  * clamp to [-128, 127]. */
 int8_t pqgo_int8_encode(float t) {
@@ -211,6 +229,26 @@ uint8_t pqgo_e2m1_encode(float t) {
         int mant = (int)(r / ldexp(1.0, Er - 1)) - 2;
         return (uint8_t)(sign | ((Er + 1) << 1) | mant);
     }
+}
+
+/* ------------------------------------------------------------------------ */
+/* NVFP4 block scale ([FI] section 6, block_size = 16; steps as listed in the */
+/* header comment)                                                          */
+/* ------------------------------------------------------------------------ */
+
+/* E4M3 block-scale code of a block with absmax `amax` (floored at EPS) under
+ * the global scale g: r = (amax / 6) * g in fp32, then the nearest E4M3 value,
+ * saturating at 448. */
+uint8_t pqgo_nvfp4_block_scale(float amax, float g) {
+    float r = (amax / PQGO_FMAX_E2M1) * g;
+    return pqgo_e4m3_encode(r);
+}
+
+/* Multiplier that takes a block's values to E2M1 units: g / value(sf) in fp32,
+ * or 0 for a zero block scale (every code of the block is then a zero). */
+float pqgo_nvfp4_multiplier(uint8_t sf, float g) {
+    float d = pqgo_e4m3_decode(sf);
+    return d == 0.0f ? 0.0f : g / d;
 }
 
 /* ------------------------------------------------------------------------ */
@@ -362,6 +400,75 @@ int pqgo_quant(const uint16_t *in, uint8_t *out, void *scales, int64_t E,
     return status;
 }
 
+/* NVFP4 quantization of E experts of M rows of K outputs (K a multiple of 16).
+ *   in, masked_m, fused: as for pqgo_quant.
+ *   out    : [E][M][K/2] bytes of E2M1 code pairs (element 2i in bits 0-3).
+ *   scales : one E4M3 byte per block of 16, layout PQGO_ROW ([E][M][K/16]),
+ *            PQGO_COL ([E][K/16][M_pad]) or PQGO_TILE128X4 (as for MXFP4).
+ *   g      : the global scale (finite, > 0).
+ * Returns 0, -1 for an invalid argument, -2 for a non-finite input value. */
+int pqgo_quant_nvfp4(const uint16_t *in, uint8_t *out, uint8_t *scales, int64_t E,
+                     int64_t M, int64_t K, int in_fp16, int layout, int fused,
+                     const int32_t *masked_m, float g) {
+    const int G = PQGO_NVFP4_BLOCK;
+    if (E < 1 || M < 0 || K <= 0 || K % G != 0) return -1;
+    if (layout != PQGO_ROW && layout != PQGO_COL && layout != PQGO_TILE128X4) return -1;
+    if (!(g > 0.0f) || !isfinite(g)) return -1;
+
+    const int64_t ng = K / G;
+    const int64_t in_width = fused ? 2 * K : K;
+    const int64_t mpad = padded_rows(M);
+    const int64_t plane = ((M + 127) / 128) * ((ng + 3) / 4) * 512;
+    float v[PQGO_NVFP4_BLOCK];
+
+    for (int64_t e = 0; e < E; ++e) {
+        int64_t rows = M;
+        if (masked_m) {
+            rows = masked_m[e];
+            if (rows < 0) rows = 0;
+            if (rows > M) rows = M;
+        }
+        for (int64_t m = 0; m < rows; ++m) {
+            const uint16_t *xrow = in + (e * M + m) * in_width;
+            uint8_t *qrow = out + (e * M + m) * (K / 2);
+            for (int64_t b = 0; b < ng; ++b) {
+                /* 1. decode (and fuse) the block's 16 values */
+                for (int i = 0; i < G; ++i) {
+                    float x = pqgo_decode(xrow[b * G + i], in_fp16);
+                    if (fused) {
+                        float up = pqgo_decode(xrow[K + b * G + i], in_fp16);
+                        if (!isfinite(x) || !isfinite(up)) return -2;
+                        x = pqgo_silu_mul(x, up);
+                    }
+                    if (!isfinite(x)) return -2;
+                    v[i] = x;
+                }
+                /* 2. absmax, 3. block scale and its multiplier */
+                float amax = pqgo_group_amax(v, G);
+                uint8_t sf = pqgo_nvfp4_block_scale(amax, g);
+                float mult = pqgo_nvfp4_multiplier(sf, g);
+                /* 4. codes, two per byte */
+                for (int i = 0; i < G; i += 2) {
+                    uint8_t lo = pqgo_e2m1_encode(v[i] * mult);
+                    uint8_t hi = pqgo_e2m1_encode(v[i + 1] * mult);
+                    qrow[(b * G + i) / 2] = (uint8_t)(lo | (hi << 4));
+                }
+                /* 5. block-scale byte */
+                if (layout == PQGO_ROW)
+                    scales[(e * M + m) * ng + b] = sf;
+                else if (layout == PQGO_COL)
+                    scales[e * ng * mpad + b * mpad + m] = sf;
+                else
+                    scales[e * plane + tile128x4_offset(m, b, ng)] = sf;
+            }
+            if (layout == PQGO_TILE128X4)
+                for (int64_t b = ng; b % 4 != 0; ++b)
+                    scales[e * plane + tile128x4_offset(m, b, ng)] = 0;
+        }
+    }
+    return 0;
+}
+
 /* ------------------------------------------------------------------------ */
 /* Array forms of the element functions, for the pin tests                   */
 /* ------------------------------------------------------------------------ */
@@ -396,4 +503,16 @@ void pqgo_ue8m0_exponent_n(const float *amax, uint8_t *e, int64_t n) {
 
 void pqgo_scale_fp32_n(const float *amax, float *s, int64_t n, int out_int8) {
     for (int64_t i = 0; i < n; ++i) s[i] = pqgo_scale_fp32(amax[i], out_int8);
+}
+
+void pqgo_e4m3_decode_n(const uint8_t *c, float *v, int64_t n) {
+    for (int64_t i = 0; i < n; ++i) v[i] = pqgo_e4m3_decode(c[i]);
+}
+
+void pqgo_nvfp4_block_scale_n(const float *amax, uint8_t *sf, int64_t n, float g) {
+    for (int64_t i = 0; i < n; ++i) sf[i] = pqgo_nvfp4_block_scale(amax[i], g);
+}
+
+void pqgo_nvfp4_multiplier_n(const uint8_t *sf, float *m, int64_t n, float g) {
+    for (int64_t i = 0; i < n; ++i) m[i] = pqgo_nvfp4_multiplier(sf[i], g);
 }

@@ -31,17 +31,24 @@ bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p
 // and returns the bytes of one expert's scale plane through *plane.
 int check_geometry(int64_t num_experts, int64_t M, int64_t K, int group, int scale_fmt,
                    int scale_layout, int64_t *plane) {
-    if (scale_fmt != PQG_SCALE_FP32 && scale_fmt != PQG_SCALE_UE8M0) return PQG_ERR_INVALID_ARG;
+    if (scale_fmt != PQG_SCALE_FP32 && scale_fmt != PQG_SCALE_UE8M0 &&
+        scale_fmt != PQG_SCALE_E4M3)
+        return PQG_ERR_INVALID_ARG;
     if (scale_layout != PQG_ROW_MAJOR && scale_layout != PQG_COL_MAJOR_TMA &&
         scale_layout != PQG_UE8M0_PACKED && scale_layout != PQG_UE8M0_TILED_128x4)
         return PQG_ERR_INVALID_ARG;
     if (group <= 0) return PQG_ERR_INVALID_ARG;
-    // G in {32, 64, 128}, or one group per row (per-token, K <= 16384)
-    const bool per_token = group == K && K % 16 == 0 && K <= kMaxPerTokenK;
-    if (group != 32 && group != 64 && group != 128 && !per_token) return PQG_ERR_UNSUPPORTED;
-    if ((scale_layout == PQG_UE8M0_PACKED || scale_layout == PQG_UE8M0_TILED_128x4) &&
-        scale_fmt != PQG_SCALE_UE8M0)
-        return PQG_ERR_UNSUPPORTED;
+    if (scale_fmt == PQG_SCALE_E4M3) {
+        // NVFP4: blocks of 16, byte scales, no packed words
+        if (group != 16 || scale_layout == PQG_UE8M0_PACKED) return PQG_ERR_UNSUPPORTED;
+    } else {
+        // G in {32, 64, 128}, or one group per row (per-token, K <= 16384)
+        const bool per_token = group == K && K % 16 == 0 && K <= kMaxPerTokenK;
+        if (group != 32 && group != 64 && group != 128 && !per_token) return PQG_ERR_UNSUPPORTED;
+        if ((scale_layout == PQG_UE8M0_PACKED || scale_layout == PQG_UE8M0_TILED_128x4) &&
+            scale_fmt != PQG_SCALE_UE8M0)
+            return PQG_ERR_UNSUPPORTED;
+    }
     if (num_experts < 1 || num_experts > static_cast<int64_t>(pqg::kMaxExperts))
         return PQG_ERR_INVALID_ARG;
     if (M < 0 || K <= 0 || K % group != 0) return PQG_ERR_INVALID_ARG;
@@ -53,7 +60,7 @@ int check_geometry(int64_t num_experts, int64_t M, int64_t K, int group, int sca
     if (M * K > (int64_t{1} << 40) / num_experts) return PQG_ERR_INVALID_ARG;
 
     const int64_t ng = K / group;
-    const int64_t elem = scale_fmt == PQG_SCALE_UE8M0 ? 1 : 4;
+    const int64_t elem = scale_fmt == PQG_SCALE_FP32 ? 4 : 1;
     if (scale_layout == PQG_ROW_MAJOR)
         *plane = M * ng * elem;
     else if (scale_layout == PQG_COL_MAJOR_TMA)
@@ -86,34 +93,30 @@ int sm_count(int device) {
 }
 }  // namespace pqg
 
-extern "C" {
+namespace {
 
-int64_t pqg_scales_bytes(int64_t num_experts, int64_t M, int64_t K, int group, int scale_fmt,
-                         int scale_layout) {
-    int64_t plane = 0;
-    const int st = check_geometry(num_experts, M, K, group, scale_fmt, scale_layout, &plane);
-    if (st != PQG_OK) return st;
-    return plane * num_experts;
-}
-
-int pqg_quant(const void *in, void *out, void *scales, int64_t M, int64_t num_experts, int64_t K,
-              int group, int in_dtype, int out_dtype, int scale_fmt, int scale_layout,
-              int fuse_silu_mul, const int32_t *masked_m, int64_t expected_m,
-              pqg_stream_t stream) {
+// Validation and launch shared by pqg_quant and pqg_quant_nvfp4.
+int quant_impl(const void *in, void *out, void *scales, const float *global_scale, int64_t M,
+               int64_t num_experts, int64_t K, int group, int in_dtype, int out_dtype,
+               int scale_fmt, int scale_layout, int fuse_silu_mul, const int32_t *masked_m,
+               int64_t expected_m, pqg_stream_t stream) {
     if (in_dtype != PQG_BF16 && in_dtype != PQG_FP16) return PQG_ERR_INVALID_ARG;
     if (out_dtype != PQG_E4M3 && out_dtype != PQG_INT8 && out_dtype != PQG_E2M1)
         return PQG_ERR_INVALID_ARG;
     int64_t plane = 0;
     const int st = check_geometry(num_experts, M, K, group, scale_fmt, scale_layout, &plane);
     if (st != PQG_OK) return st;
+    const bool nvfp4 = scale_fmt == PQG_SCALE_E4M3;
     if (scale_fmt == PQG_SCALE_UE8M0 && out_dtype == PQG_INT8) return PQG_ERR_UNSUPPORTED;
-    if (out_dtype == PQG_E2M1 &&
+    if (out_dtype == PQG_E2M1 && !nvfp4 &&
         (scale_fmt != PQG_SCALE_UE8M0 || (group != 32 && group != 64 && group != 128)))
         return PQG_ERR_UNSUPPORTED;  // MXFP4: UE8M0 scales, groups of 32/64/128
     if (M == 0) return PQG_OK;
 
     if (in == nullptr || out == nullptr || scales == nullptr) return PQG_ERR_INVALID_ARG;
+    if (nvfp4 && global_scale == nullptr) return PQG_ERR_INVALID_ARG;
     if (!aligned(in, 32) || !aligned(out, 16)) return PQG_ERR_ALIGNMENT;
+    if (nvfp4 && !aligned(global_scale, 4)) return PQG_ERR_ALIGNMENT;
     if (scale_fmt == PQG_SCALE_FP32 || scale_layout == PQG_UE8M0_PACKED) {
         if (!aligned(scales, 4)) return PQG_ERR_ALIGNMENT;
     }
@@ -132,6 +135,7 @@ int pqg_quant(const void *in, void *out, void *scales, int64_t M, int64_t num_ex
     a.p.out = static_cast<uint8_t *>(out);
     a.p.scales = static_cast<uint8_t *>(scales);
     a.p.masked_m = masked_m;
+    a.p.gscale = global_scale;
     a.p.in_expert_bytes = M * in_row_bytes;
     a.p.out_expert_bytes = M * out_row_bytes;
     a.p.out_row_bytes = static_cast<uint32_t>(out_row_bytes);
@@ -149,7 +153,8 @@ int pqg_quant(const void *in, void *out, void *scales, int64_t M, int64_t num_ex
     a.expected_strips = static_cast<uint64_t>(num_experts * grid_rows) * a.p.segs;
     a.expected_rows = static_cast<uint64_t>(num_experts * grid_rows);
     a.group = group;
-    a.kind = out_dtype == PQG_E2M1           ? pqg::Kind::E2M1_UE8M0
+    a.kind = nvfp4                            ? pqg::Kind::E2M1_E4M3
+             : out_dtype == PQG_E2M1          ? pqg::Kind::E2M1_UE8M0
              : scale_fmt == PQG_SCALE_UE8M0 ? pqg::Kind::E4M3_UE8M0
              : out_dtype == PQG_INT8        ? pqg::Kind::INT8_FP32
                                             : pqg::Kind::E4M3_FP32;
@@ -165,6 +170,36 @@ int pqg_quant(const void *in, void *out, void *scales, int64_t M, int64_t num_ex
     }
     g_launches.fetch_add(1, std::memory_order_relaxed);
     return PQG_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int64_t pqg_scales_bytes(int64_t num_experts, int64_t M, int64_t K, int group, int scale_fmt,
+                         int scale_layout) {
+    int64_t plane = 0;
+    const int st = check_geometry(num_experts, M, K, group, scale_fmt, scale_layout, &plane);
+    if (st != PQG_OK) return st;
+    return plane * num_experts;
+}
+
+int pqg_quant(const void *in, void *out, void *scales, int64_t M, int64_t num_experts, int64_t K,
+              int group, int in_dtype, int out_dtype, int scale_fmt, int scale_layout,
+              int fuse_silu_mul, const int32_t *masked_m, int64_t expected_m,
+              pqg_stream_t stream) {
+    if (scale_fmt == PQG_SCALE_E4M3) return PQG_ERR_UNSUPPORTED;  // pqg_quant_nvfp4
+    return quant_impl(in, out, scales, nullptr, M, num_experts, K, group, in_dtype, out_dtype,
+                      scale_fmt, scale_layout, fuse_silu_mul, masked_m, expected_m, stream);
+}
+
+int pqg_quant_nvfp4(const void *in, void *out, void *scales, const float *global_scale,
+                    int64_t M, int64_t num_experts, int64_t K, int in_dtype, int scale_layout,
+                    int fuse_silu_mul, const int32_t *masked_m, int64_t expected_m,
+                    pqg_stream_t stream) {
+    return quant_impl(in, out, scales, global_scale, M, num_experts, K, 16, in_dtype, PQG_E2M1,
+                      PQG_SCALE_E4M3, scale_layout, fuse_silu_mul, masked_m, expected_m,
+                      stream);
 }
 
 const char *pqg_status_string(int status) {

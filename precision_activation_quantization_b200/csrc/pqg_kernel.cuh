@@ -22,8 +22,9 @@
 // Memory-level parallelism.  A warp takes ITEMS strips per chunk and issues
 // all of the chunk's 32-byte loads before any arithmetic; with about 40
 // resident warps per SM (register-light kernel) that keeps the HBM queues full.
-// Keeping a second chunk in flight (register double-buffering) was measured
-// slower: the extra registers cost more warps than the prefetch won.
+// Keeping a second chunk in flight was measured slower both ways it was tried:
+// in registers (double-buffering) and in shared memory (cp.async stages), the
+// extra registers and instructions cost more warps than the prefetch won.
 //
 // Exact division.  Codes must equal a rounding of fp32(x / s).  A per-element
 // IEEE division is too slow for a bandwidth-bound loop, so the quotient is
@@ -53,11 +54,22 @@
 
 namespace pqg {
 
-enum class Kind : int { E4M3_FP32 = 0, E4M3_UE8M0 = 1, INT8_FP32 = 2, E2M1_UE8M0 = 3 };
+// E2M1_UE8M0 is MXFP4 (G = 32/64/128); E2M1_E4M3 is NVFP4 (G = 16, an E4M3
+// block scale under a per-call fp32 global scale).
+enum class Kind : int { E4M3_FP32 = 0, E4M3_UE8M0 = 1, INT8_FP32 = 2, E2M1_UE8M0 = 3,
+                        E2M1_E4M3 = 4 };
 
 // Kinds whose scale is a UE8M0 power of two.
 __host__ __device__ constexpr bool is_ue8m0(Kind k) {
     return k == Kind::E4M3_UE8M0 || k == Kind::E2M1_UE8M0;
+}
+// Kinds with FP4 codes, two per byte.
+__host__ __device__ constexpr bool is_e2m1(Kind k) {
+    return k == Kind::E2M1_UE8M0 || k == Kind::E2M1_E4M3;
+}
+// Kinds whose stored scale is one byte (UE8M0 exponent or E4M3 block scale).
+__host__ __device__ constexpr bool byte_scale(Kind k) {
+    return is_ue8m0(k) || k == Kind::E2M1_E4M3;
 }
 
 // Runtime scale layouts (same numbering as the C ABI's pqg_scale_layout).
@@ -88,6 +100,7 @@ struct Params {
     uint8_t *out;              // expert 0, row 0
     uint8_t *scales;           // expert 0's scale plane (byte address)
     const int32_t *masked_m;   // device int32[experts], or null: all M rows
+    const float *gscale;       // NVFP4 only: device fp32 global scale g
     int64_t in_expert_bytes;   // M * in_row_bytes
     int64_t out_expert_bytes;  // M * out_row_bytes
     int64_t scale_expert_bytes;
@@ -298,17 +311,51 @@ __device__ __forceinline__ uint32_t ue8m0_exponent_e2m1(float amax) {
 }
 
 struct GroupScale {
-    float mult;   // UE8M0: 2^(127-e) (exact); fp32 kinds: y = RN(1/s)
+    float mult;   // UE8M0: 2^(127-e) (exact); fp32 kinds: y = RN(1/s); NVFP4: g / value(sf)
     float neg_s;  // fp32 kinds: -s
     float s;      // fp32 kinds: the stored scale
-    uint32_t e8;  // UE8M0: the stored exponent byte
+    uint32_t e8;  // UE8M0: the stored exponent byte; NVFP4: the E4M3 block-scale byte
 };
 
+// NVFP4 ("block_size = 16 -> NVFP4", FlashInfer GEMM notes, section 6).  Per
+// block of 16, in fp32: r = RN(amax / 6) * g, the block-scale byte sf = nearest
+// E4M3 code of r (satfinite: 448 at most), and the codes' multiplier g /
+// value(sf), 0 for sf = 0.  A block-scale code has 127 non-negative values, so
+// each CTA divides once per code into a shared-memory table (nv[0..127]; nv[128]
+// holds g) instead of once per block.  RN(amax / 6) uses div_by_const, checked
+// exhaustively against the IEEE quotient over every fp32 amax >= 1e-10.
+constexpr float kRcp6 = 0x1.555556p-3f;    // RN(1/6)
+constexpr int kNvTable = 129;
+
+__device__ __forceinline__ float e4m3_code_value(uint32_t c) {
+    // (8 + m) * 2^(e - 10) for exponent field e >= 1, m * 2^-9 for e = 0
+    const uint32_t e = (c >> 3) & 15u, m = c & 7u;
+    const float p2 = __uint_as_float((max(e, 1u) + 117u) << 23);
+    return p2 * static_cast<float>(e != 0u ? 8u + m : m);
+}
+
+// Every thread of the CTA calls it (blockDim.x >= 128); ends with __syncthreads.
+__device__ __forceinline__ void build_nvfp4_table(const Params &p, float *nv) {
+    if (threadIdx.x < 128u) {
+        const float g = __ldg(p.gscale);
+        const float d = e4m3_code_value(threadIdx.x);
+        nv[threadIdx.x] = d == 0.0f ? 0.0f : __fdiv_rn(g, d);
+        if (threadIdx.x == 0u) nv[128] = g;
+    }
+    __syncthreads();
+}
+
 template <Kind KIND>
-__device__ __forceinline__ GroupScale make_scale(float amax) {
+__device__ __forceinline__ GroupScale make_scale(float amax, const float *nv = nullptr) {
     GroupScale gs;
     amax = fmaxf(amax, 1e-10f);   // EPS floor
-    if constexpr (is_ue8m0(KIND)) {
+    if constexpr (KIND == Kind::E2M1_E4M3) {
+        const float r = __fmul_rn(div_by_const(amax, 6.0f, kRcp6), nv[128]);
+        gs.e8 = e4m3x2(r, 0.0f) & 0xFFu;
+        gs.mult = nv[gs.e8 & 0x7Fu];   // r >= 0: the sign bit is clear
+        gs.s = 0.0f;
+        gs.neg_s = 0.0f;
+    } else if constexpr (is_ue8m0(KIND)) {
         gs.e8 = KIND == Kind::E2M1_UE8M0 ? ue8m0_exponent_e2m1(amax) : ue8m0_exponent(amax);
         gs.mult = __uint_as_float((254u - gs.e8) << 23);
         gs.s = 0.0f;
@@ -327,7 +374,7 @@ __device__ __forceinline__ GroupScale make_scale(float amax) {
 template <Kind KIND>
 __device__ __forceinline__ void encode16(const float (&v)[16], const GroupScale &gs,
                                          uint32_t (&w)[4]) {
-    if constexpr (KIND == Kind::E2M1_UE8M0) {
+    if constexpr (is_e2m1(KIND)) {
         // 16 codes in 8 bytes: w[0] elements 0..7, w[1] elements 8..15
         const float2 m2 = make_float2(gs.mult, gs.mult);
 #pragma unroll
@@ -569,7 +616,7 @@ __device__ __forceinline__ void load_chunk(Chunk<ITEMS, FUSED> &ch, uint32_t s, 
 template <typename In, int G, Kind KIND, bool FUSED>
 __device__ __forceinline__ void quantize_strip(const uint32_t (&x)[8], const uint32_t *u,
                                                uint32_t e, uint32_t row, uint32_t col,
-                                               const Params &p, uint32_t lane) {
+                                               const Params &p, uint32_t lane, const float *nv) {
     constexpr int L = G / 16;  // lanes per group
     const bool ok = col < p.K;
     const uint32_t g = col / G;  // group within the row (valid lanes)
@@ -624,7 +671,7 @@ __device__ __forceinline__ void quantize_strip(const uint32_t (&x)[8], const uin
         for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
 #pragma unroll
         for (int o = 1; o < L; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
-        gs = make_scale<KIND>(amax);
+        gs = make_scale<KIND>(amax, nv);
         encode16<KIND>(v, gs, w);
     }
 
@@ -639,7 +686,7 @@ __device__ __forceinline__ void quantize_strip(const uint32_t (&x)[8], const uin
     if (!ok) return;
 
     uint8_t *dst = p.out + e * p.out_expert_bytes + static_cast<uint64_t>(row) * p.out_row_bytes;
-    if constexpr (KIND == Kind::E2M1_UE8M0)
+    if constexpr (is_e2m1(KIND))
         store8B(dst + col / 2u, w[0], w[1]);
     else
         store16B(dst + col, w[0], w[1], w[2], w[3]);
@@ -654,7 +701,7 @@ __device__ __forceinline__ void quantize_strip(const uint32_t (&x)[8], const uin
         } else {
             const uint64_t idx = (p.layout == kRowMajor) ? static_cast<uint64_t>(row) * p.ng + g
                                                          : static_cast<uint64_t>(g) * p.mpad + row;
-            if constexpr (is_ue8m0(KIND))
+            if constexpr (byte_scale(KIND))
                 sc[idx] = static_cast<uint8_t>(gs.e8);
             else
                 reinterpret_cast<float *>(sc)[idx] = gs.s;
@@ -664,12 +711,12 @@ __device__ __forceinline__ void quantize_strip(const uint32_t (&x)[8], const uin
 
 template <typename In, int G, Kind KIND, bool FUSED, int ITEMS>
 __device__ __forceinline__ void quantize_chunk(const Chunk<ITEMS, FUSED> &ch, const Params &p,
-                                               uint32_t lane) {
+                                               uint32_t lane, const float *nv) {
 #pragma unroll
     for (int k = 0; k < ITEMS; ++k) {
         if (static_cast<uint32_t>(k) >= ch.n) break;  // warp-uniform
         quantize_strip<In, G, KIND, FUSED>(ch.x[k], FUSED ? ch.u[k] : nullptr, ch.e[k],
-                                           ch.row[k], ch.col[k], p, lane);
+                                           ch.row[k], ch.col[k], p, lane, nv);
     }
 }
 
@@ -678,25 +725,36 @@ __device__ __forceinline__ void quantize_chunk(const Chunk<ITEMS, FUSED> &ch, co
 // ---------------------------------------------------------------------------
 
 // Resident CTAs per SM the register allocation must allow (0: no constraint).
-// The fp32-scale plain variants run best at 5 (<= 51 registers); the rest need
-// no constraint.
+// The fp32-scale plain variants run best at 5 (<= 51 registers) and flat NVFP4
+// at 6 (<= 40 registers, no spills); the rest need no constraint.
 #ifndef PQG_MIN_BLOCKS_FP32
 #define PQG_MIN_BLOCKS_FP32 5
 #endif
-template <Kind KIND, bool FUSED>
+#ifndef PQG_MIN_BLOCKS_NVFP4
+#define PQG_MIN_BLOCKS_NVFP4 6
+#endif
+template <Kind KIND, bool FUSED, bool MULTI>
 constexpr int min_blocks() {
-    return (!is_ue8m0(KIND) && !FUSED) ? PQG_MIN_BLOCKS_FP32 : 0;
+    if constexpr (FUSED) return 0;
+    if constexpr (KIND == Kind::E4M3_FP32 || KIND == Kind::INT8_FP32) return PQG_MIN_BLOCKS_FP32;
+    if constexpr (KIND == Kind::E2M1_E4M3 && !MULTI) return PQG_MIN_BLOCKS_NVFP4;
+    return 0;
 }
 
 template <typename In, int G, Kind KIND, bool FUSED, int ITEMS, int WARPS, bool MULTI>
-__global__ void __launch_bounds__(WARPS * 32, min_blocks<KIND, FUSED>())
+__global__ void __launch_bounds__(WARPS * 32, min_blocks<KIND, FUSED, MULTI>())
     quant_kernel(const __grid_constant__ Params p) {
-    static_assert(G == 32 || G == 64 || G == 128, "G must be 32, 64 or 128");
+    static_assert((G == 32 || G == 64 || G == 128) == (KIND != Kind::E2M1_E4M3) &&
+                      (G == 16) == (KIND == Kind::E2M1_E4M3),
+                  "G is 32, 64 or 128, or 16 for NVFP4");
+    static_assert(WARPS * 32 >= 128, "the NVFP4 table is built by 128 threads");
     extern __shared__ __align__(16) uint32_t smem_prefix[];
+    __shared__ float nv[KIND == Kind::E2M1_E4M3 ? kNvTable : 1];
 
     wait_for_producer();                        // before the first global access
     const uint32_t lane = threadIdx.x & 31u;
     const uint32_t warp = threadIdx.x >> 5;
+    if constexpr (KIND == Kind::E2M1_E4M3) build_nvfp4_table(p, nv);
     ExpertTable t;
     if constexpr (MULTI) {
         t = make_table(p, smem_prefix, lane);
@@ -716,7 +774,7 @@ __global__ void __launch_bounds__(WARPS * 32, min_blocks<KIND, FUSED>())
         if (s >= t.total) break;                // warp-uniform
         Chunk<ITEMS, FUSED> ch;
         load_chunk<ITEMS, FUSED, MULTI>(ch, s, min(items, t.total - s), t, p, lane);
-        quantize_chunk<In, G, KIND, FUSED, ITEMS>(ch, p, lane);
+        quantize_chunk<In, G, KIND, FUSED, ITEMS>(ch, p, lane, nv);
     }
     release_dependents();
 }

@@ -64,18 +64,20 @@ cudaError_t launch_variant(const LaunchArgs &a) {
     constexpr int kThreads = Sh::kWarps * 32;
     auto kernel = quant_kernel<In, G, KIND, FUSED, Sh::kItems, Sh::kWarps, MULTI>;
 
-    // Resident CTAs per SM, queried once per variant for the largest expert
-    // table (16 KB of shared memory); registers are the binding limit.
-    static const int blocks_per_sm = [&] {
-        int n = 0;
+    // Resident CTAs per SM, queried once per variant without and with the
+    // largest shared-memory expert table (more than 32 experts).
+    static const int2 occupancy = [&] {
+        int n0 = 0, n1 = 0;
         if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  static_cast<int>(smem_bytes(kMaxExperts))) != cudaSuccess ||
-            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, kThreads,
-                                                          smem_bytes(kMaxExperts)) != cudaSuccess ||
-            n < 1)
-            n = 1;
-        return n;
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n0, kernel, kThreads, 0) !=
+                cudaSuccess ||
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n1, kernel, kThreads,
+                                                          smem_bytes(kMaxExperts)) != cudaSuccess)
+            n0 = n1 = 1;
+        return make_int2(n0 < 1 ? 1 : n0, n1 < 1 ? 1 : n1);
     }();
+    const int blocks_per_sm = smem_bytes(a.p.experts) == 0 ? occupancy.x : occupancy.y;
 
     int device = 0;
     cudaError_t err = cudaGetDevice(&device);
@@ -127,6 +129,7 @@ cudaError_t launch_group(const LaunchArgs &a) {
         case Kind::E4M3_UE8M0: return launch_kind<In, G, Kind::E4M3_UE8M0>(a);
         case Kind::INT8_FP32: return launch_kind<In, G, Kind::INT8_FP32>(a);
         case Kind::E2M1_UE8M0: return launch_kind<In, G, Kind::E2M1_UE8M0>(a);
+        case Kind::E2M1_E4M3: break;  // G = 16 only (launch_dtype)
     }
     return cudaErrorInvalidValue;
 }
@@ -216,13 +219,16 @@ cudaError_t launch_row(const LaunchArgs &a) {
             return a.fused ? launch_row_kind<In, Kind::INT8_FP32, true>(a)
                            : launch_row_kind<In, Kind::INT8_FP32, false>(a);
         case Kind::E2M1_UE8M0:
-            break;  // rejected by the caller: MXFP4 groups are 32/64/128 wide
+        case Kind::E2M1_E4M3:
+            break;  // rejected by the caller: FP4 groups are 16 (NVFP4) or 32/64/128
     }
     return cudaErrorInvalidValue;
 }
 
 template <typename In>
 cudaError_t launch_dtype(const LaunchArgs &a) {
+    if (a.kind == Kind::E2M1_E4M3)
+        return a.group == 16 ? launch_kind<In, 16, Kind::E2M1_E4M3>(a) : cudaErrorInvalidValue;
     switch (a.group) {
         case 32: return launch_group<In, 32>(a);
         case 64: return launch_group<In, 64>(a);

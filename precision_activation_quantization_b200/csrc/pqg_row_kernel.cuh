@@ -25,7 +25,7 @@ constexpr int kRowThreads = 256;  // 8 warps per CTA
 template <typename In, Kind KIND, bool FUSED, int SLOTS>
 __global__ void __launch_bounds__(kRowThreads)
     row_quant_kernel(const __grid_constant__ Params p) {
-    static_assert(KIND != Kind::E2M1_UE8M0, "per-token E2M1 is not offered");
+    static_assert(!is_e2m1(KIND), "per-token E2M1 is not offered");
     extern __shared__ __align__(16) uint32_t smem_prefix[];
     __shared__ float partial[2][kRowThreads / 32];
 

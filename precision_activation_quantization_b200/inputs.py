@@ -92,6 +92,7 @@ class Workload:
     fused: bool = False
     masked_m: np.ndarray | None = None   # int32 [E] or None (flat)
     expected_m: int = 0
+    global_scale: float | None = None    # NVFP4 (scale_fmt "e4m3") only
 
     @property
     def rows(self) -> int:
@@ -112,8 +113,10 @@ class Workload:
         if self.layout in ("packed", "tile128x4"):
             scale_row = 4 * ((ng + 3) // 4)
         else:
-            scale_row = ng * (1 if self.scale_fmt == "ue8m0" else 4)
+            scale_row = ng * (4 if self.scale_fmt == "fp32" else 1)
         extra = 0 if self.masked_m is None else 4 * self.E
+        if self.global_scale is not None:
+            extra += 4                   # the fp32 global scale
         return self.rows * (in_row + out_row + scale_row) + extra
 
     def with_(self, **kw) -> "Workload":
@@ -188,6 +191,20 @@ def mxfp4(M: int = 8192, K: int = 7168, seed: int = 1) -> Workload:
     scales in the 128x4 tiled layout."""
     w = flat_hidden(M=M, K=K, seed=seed)
     return w.with_(name=f"mxfp4_{M}x{K}", group=32, out_dtype="e2m1", layout="tile128x4")
+
+
+# 448 * 6 / 1024: the global scale of a tensor whose absmax is about 1024 (the
+# hidden-state input's x200 outliers reach a few hundred to about a thousand)
+NVFP4_GLOBAL_SCALE = 2.625
+
+
+def nvfp4(M: int = 8192, K: int = 7168, seed: int = 1,
+          global_scale: float = NVFP4_GLOBAL_SCALE) -> Workload:
+    """The flat hidden-state input as an NVFP4 operand: blocks of 16, E2M1 codes,
+    E4M3 block scales in the 128x4 tiled layout, a fixed fp32 global scale."""
+    w = flat_hidden(M=M, K=K, seed=seed)
+    return w.with_(name=f"nvfp4_{M}x{K}", group=16, out_dtype="e2m1", scale_fmt="e4m3",
+                   layout="tile128x4", global_scale=global_scale)
 
 
 def sweep(M: int, K: int = 4096, in_dtype: str = "bf16", group: int = 128,

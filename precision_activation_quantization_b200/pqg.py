@@ -28,17 +28,17 @@ PQG_ERR_ALIGNMENT = -3
 PQG_ERR_CUDA = -4
 
 PQG_BF16, PQG_FP16, PQG_E4M3, PQG_INT8, PQG_E2M1 = 0, 1, 2, 3, 4
-PQG_SCALE_FP32, PQG_SCALE_UE8M0 = 0, 1
+PQG_SCALE_FP32, PQG_SCALE_UE8M0, PQG_SCALE_E4M3 = 0, 1, 2
 PQG_ROW_MAJOR, PQG_COL_MAJOR_TMA, PQG_UE8M0_PACKED, PQG_UE8M0_TILED_128x4 = 0, 1, 2, 3
 
 IN_DTYPES = {"bf16": PQG_BF16, "fp16": PQG_FP16}
 OUT_DTYPES = {"e4m3": PQG_E4M3, "int8": PQG_INT8, "e2m1": PQG_E2M1}
-SCALE_FMTS = {"fp32": PQG_SCALE_FP32, "ue8m0": PQG_SCALE_UE8M0}
+SCALE_FMTS = {"fp32": PQG_SCALE_FP32, "ue8m0": PQG_SCALE_UE8M0, "e4m3": PQG_SCALE_E4M3}
 LAYOUTS = {"row": PQG_ROW_MAJOR, "col": PQG_COL_MAJOR_TMA, "packed": PQG_UE8M0_PACKED,
            "tile128x4": PQG_UE8M0_TILED_128x4}
 
-EXPORTS = ("pqg_quant", "pqg_scales_bytes", "pqg_status_string", "pqg_last_cuda_error",
-           "pqg_set_pdl", "pqg_launch_count", "pqg_version")
+EXPORTS = ("pqg_quant", "pqg_quant_nvfp4", "pqg_scales_bytes", "pqg_status_string",
+           "pqg_last_cuda_error", "pqg_set_pdl", "pqg_launch_count", "pqg_version")
 
 
 class PqgError(RuntimeError):
@@ -57,6 +57,8 @@ def _load() -> ctypes.CDLL:
     lib.pqg_quant.restype = i32
     lib.pqg_quant.argtypes = [vp, vp, vp, i64, i64, i64, i32, i32, i32, i32, i32, i32, vp,
                               i64, vp]
+    lib.pqg_quant_nvfp4.restype = i32
+    lib.pqg_quant_nvfp4.argtypes = [vp, vp, vp, vp, i64, i64, i64, i32, i32, i32, vp, i64, vp]
     lib.pqg_scales_bytes.restype = i64
     lib.pqg_scales_bytes.argtypes = [i64, i64, i64, i32, i32, i32]
     lib.pqg_status_string.restype = ctypes.c_char_p
@@ -85,6 +87,15 @@ def pqg_quant(in_ptr: int, out_ptr: int, scales_ptr: int, M: int, num_experts: i
     return _lib.pqg_quant(in_ptr, out_ptr, scales_ptr, M, num_experts, K, group, in_dtype,
                           out_dtype, scale_fmt, scale_layout, fuse_silu_mul, masked_m_ptr,
                           expected_m, stream)
+
+
+def pqg_quant_nvfp4(in_ptr: int, out_ptr: int, scales_ptr: int, global_scale_ptr: int, M: int,
+                    num_experts: int, K: int, in_dtype: int, scale_layout: int,
+                    fuse_silu_mul: int, masked_m_ptr: int | None, expected_m: int,
+                    stream: int | None) -> int:
+    return _lib.pqg_quant_nvfp4(in_ptr, out_ptr, scales_ptr, global_scale_ptr, M, num_experts,
+                                K, in_dtype, scale_layout, fuse_silu_mul, masked_m_ptr,
+                                expected_m, stream)
 
 
 def pqg_scales_bytes(num_experts: int, M: int, K: int, group: int, scale_fmt: int,
@@ -136,7 +147,7 @@ def scales_spec(M: int, K: int, group: int, scale_fmt: str = "fp32", layout: str
         return (num_experts, (M + 127) // 128 * ((ng + 3) // 4) * 512), torch.uint8
     else:
         return (num_experts, (ng + 3) // 4, mpad), torch.int32
-    return shape, (torch.uint8 if scale_fmt == "ue8m0" else torch.float32)
+    return shape, (torch.float32 if scale_fmt == "fp32" else torch.uint8)
 
 
 def allocate_outputs(M: int, K: int, group: int, *, num_experts: int = 1,
@@ -176,11 +187,13 @@ def infer_scale_layout(scales, M: int, K: int, group: int) -> str:
 def quant(x, out=None, scales=None, *, M: int | None = None, K: int | None = None,
           group: int = 128, num_experts: int | None = None, out_dtype: str = "e4m3",
           scale_fmt: str = "fp32", layout: str = "row", fuse_silu_mul: bool = False,
-          masked_m=None, expected_m: int = 0, stream=None):
+          masked_m=None, expected_m: int = 0, global_scale=None, stream=None):
     """Quantize a CUDA tensor; returns (out, scales).
 
     ``x`` is bf16/fp16, [E, M, K] / [M, K] ([..., 2K] when ``fuse_silu_mul``).
     ``masked_m`` is an int32 CUDA tensor of E row counts (masked dispatch).
+    NVFP4 is ``out_dtype="e2m1", scale_fmt="e4m3", group=16`` with
+    ``global_scale`` a one-element fp32 CUDA tensor (pqg_quant_nvfp4).
     The kernel runs on ``stream`` (default: torch's current stream).
     """
     import torch
@@ -220,6 +233,19 @@ def quant(x, out=None, scales=None, *, M: int | None = None, K: int | None = Non
         mm_ptr = masked_m.data_ptr()
     if stream is None:
         stream = torch.cuda.current_stream(x.device)
+    if scale_fmt == "e4m3":
+        if (global_scale is None or global_scale.dtype != torch.float32
+                or global_scale.numel() != 1 or global_scale.device != x.device):
+            raise ValueError("NVFP4 needs global_scale: a one-element fp32 tensor on x's device")
+        if out_dtype != "e2m1" or group != 16:
+            raise ValueError("scale_fmt='e4m3' is NVFP4: out_dtype='e2m1', group=16")
+        st = pqg_quant_nvfp4(x.data_ptr(), out.data_ptr(), scales.data_ptr(),
+                             global_scale.data_ptr(), M, E, K, in_dtype, LAYOUTS[layout],
+                             int(bool(fuse_silu_mul)), mm_ptr, int(expected_m),
+                             getattr(stream, "cuda_stream", stream))
+        if st != PQG_OK:
+            raise PqgError(st, "pqg_quant_nvfp4")
+        return out, scales
     st = pqg_quant(x.data_ptr(), out.data_ptr(), scales.data_ptr(), M, E, K, group, in_dtype,
                    OUT_DTYPES[out_dtype], SCALE_FMTS[scale_fmt], LAYOUTS[layout],
                    int(bool(fuse_silu_mul)), mm_ptr, int(expected_m),

@@ -23,7 +23,8 @@ def _torch_input(w):
 
 
 def run_gpu(w, *, expected_m=None, stream=None, x_dev=None):
-    """Run ``w`` through pqg_quant; returns (codes uint8 [E*M*K], scale bytes)."""
+    """Run ``w`` through pqg_quant (pqg_quant_nvfp4 for E4M3 block scales);
+    returns (codes uint8 [E*M*K], scale bytes)."""
     x = _torch_input(w) if x_dev is None else x_dev
     n_out = w.E * w.M * (w.K // 2 if w.out_dtype == "e2m1" else w.K)
     nbytes = pqg.pqg_scales_bytes(w.E, w.M, w.K, w.group, pqg.SCALE_FMTS[w.scale_fmt],
@@ -33,11 +34,18 @@ def run_gpu(w, *, expected_m=None, stream=None, x_dev=None):
     sc = torch.full((nbytes + GUARD,), SENTINEL, dtype=torch.uint8, device="cuda")
     mm = None if w.masked_m is None else torch.from_numpy(np.asarray(w.masked_m, np.int32)).cuda()
     s = stream if stream is not None else torch.cuda.current_stream()
-    st = pqg.pqg_quant(x.data_ptr(), out.data_ptr(), sc.data_ptr(), w.M, w.E, w.K, w.group,
-                       pqg.IN_DTYPES[w.in_dtype], pqg.OUT_DTYPES[w.out_dtype],
-                       pqg.SCALE_FMTS[w.scale_fmt], pqg.LAYOUTS[w.layout], int(w.fused),
-                       None if mm is None else mm.data_ptr(),
-                       w.expected_m if expected_m is None else expected_m, s.cuda_stream)
+    em = w.expected_m if expected_m is None else expected_m
+    if w.scale_fmt == "e4m3":
+        gsc = torch.tensor([w.global_scale], dtype=torch.float32, device="cuda")
+        st = pqg.pqg_quant_nvfp4(x.data_ptr(), out.data_ptr(), sc.data_ptr(), gsc.data_ptr(),
+                                 w.M, w.E, w.K, pqg.IN_DTYPES[w.in_dtype],
+                                 pqg.LAYOUTS[w.layout], int(w.fused),
+                                 None if mm is None else mm.data_ptr(), em, s.cuda_stream)
+    else:
+        st = pqg.pqg_quant(x.data_ptr(), out.data_ptr(), sc.data_ptr(), w.M, w.E, w.K, w.group,
+                           pqg.IN_DTYPES[w.in_dtype], pqg.OUT_DTYPES[w.out_dtype],
+                           pqg.SCALE_FMTS[w.scale_fmt], pqg.LAYOUTS[w.layout], int(w.fused),
+                           None if mm is None else mm.data_ptr(), em, s.cuda_stream)
     assert st == pqg.PQG_OK, pqg.pqg_status_string(st)
     torch.cuda.synchronize()
     out_h, sc_h = out.cpu().numpy(), sc.cpu().numpy()
@@ -50,7 +58,8 @@ def run_oracle(w):
     """The oracle's (codes uint8 [E*M*K], scale bytes), sentinel-filled like run_gpu."""
     q, s = oracle.quant(w.x, E=w.E, M=w.M, K=w.K, group=w.group, in_dtype=w.in_dtype,
                         out_dtype=w.out_dtype, scale_fmt=w.scale_fmt, layout=w.layout,
-                        fused=w.fused, masked_m=w.masked_m, fill=SENTINEL)
+                        fused=w.fused, masked_m=w.masked_m, fill=SENTINEL,
+                        global_scale=w.global_scale)
     return q.reshape(-1), s.view(np.uint8).reshape(-1)
 
 
@@ -95,10 +104,11 @@ E4M3_RANK = np.searchsorted(_FINITE, np.nan_to_num(E4M3))  # code -> position
 
 
 def _scale_planes(w, sbytes):
-    """Per-group scales as float64 [E, M, ng] from the scale buffer, and the
-    matching UE8M0 byte table (or None)."""
+    """Per-group scales as float64 [E, M, ng] from the scale buffer (for NVFP4
+    the dequantization factor value(sf) / g), and the matching byte table
+    (UE8M0 exponents or E4M3 block-scale codes; None for fp32 scales)."""
     ng, mpad = w.K // w.group, (w.M + 3) // 4 * 4
-    if w.scale_fmt == "ue8m0":
+    if w.scale_fmt != "fp32":
         if w.layout == "tile128x4":
             m = np.arange(w.M)[:, None]
             g = np.arange(ng)[None, :]
@@ -106,14 +116,15 @@ def _scale_planes(w, sbytes):
                    + ((m % 128) // 32) * 4 + g % 4)
             plane = sbytes.reshape(w.E, -1)
             e8 = plane[:, off]
-            return np.exp2(e8.astype(np.float64) - 127.0), e8
-        if w.layout == "packed":
+        elif w.layout == "packed":
             words = sbytes.reshape(w.E, (ng + 3) // 4, mpad, 4)
             e8 = words.transpose(0, 2, 1, 3).reshape(w.E, mpad, -1)[:, :w.M, :ng]
         elif w.layout == "col":
             e8 = sbytes.reshape(w.E, ng, mpad)[:, :, :w.M].transpose(0, 2, 1)
         else:
             e8 = sbytes.reshape(w.E, w.M, ng)
+        if w.scale_fmt == "e4m3":
+            return E4M3[e8] / np.float64(np.float32(w.global_scale)), e8
         return np.exp2(e8.astype(np.float64) - 127.0), e8
     f = sbytes.view(np.float32)
     if w.layout == "col":
@@ -155,7 +166,7 @@ def check_fused(w, *, max_flip_frac=1e-4, rel_tol=7e-2, **kw):
         word = idx // 4
         m_of, e_of = word % mpad, word // (((ng + 3) // 4) * mpad)
     else:
-        elem = idx // (1 if w.scale_fmt == "ue8m0" else 4)
+        elem = idx // (4 if w.scale_fmt == "fp32" else 1)
         if w.layout == "col":
             m_of, e_of = elem % mpad, elem // (ng * mpad)
         else:
@@ -175,7 +186,20 @@ def check_fused(w, *, max_flip_frac=1e-4, rel_tol=7e-2, **kw):
     amax = np.maximum(np.abs(yg).max(-1), 1e-10)
 
     g_sc, r_sc = g_sc[live], r_sc[live]                                # [n_live, ng]
-    if g_e8 is not None:
+    if g_e8 is not None and w.scale_fmt == "e4m3":
+        # NVFP4: the block-scale code may move only where amax * g / 6 lies
+        # within a few fp32 ulps of an E4M3 rounding midpoint
+        g_e8, r_e8 = g_e8[live].astype(np.int64), r_e8[live].astype(np.int64)
+        scale_diff = g_e8 != r_e8
+        r = np.minimum(amax[live] * np.float64(np.float32(w.global_scale)) / 6.0, 448.0)
+        vals = np.sort(np.unique(np.abs(E4M3[~np.isnan(E4M3)])))
+        mids = (vals[1:] + vals[:-1]) / 2.0
+        dist = np.min(np.abs(r[..., None] / mids - 1.0), axis=-1)
+        assert (~scale_diff | (dist < 2.0 ** -18)).all(), \
+            f"{w.name}: {int((scale_diff & (dist >= 2.0 ** -18)).sum())} block scales differ"
+        assert (np.abs(E4M3_RANK[g_e8] - E4M3_RANK[r_e8]) <= 1).all()
+        exempt = scale_diff
+    elif g_e8 is not None:
         g_e8, r_e8 = g_e8[live].astype(np.int64), r_e8[live].astype(np.int64)
         scale_diff = g_e8 != r_e8
         r = (amax[live] / 448.0)
@@ -211,15 +235,32 @@ def check_fused(w, *, max_flip_frac=1e-4, rel_tol=7e-2, **kw):
             else E2M1[gcodes] if w.out_dtype == "e2m1" else E4M3[gcodes])
     deq = vals * g_sc[..., None]
     yl = y[live].reshape(-1, K // G, G)
-    t = np.abs(yl) / g_sc[..., None]
+    with np.errstate(divide="ignore", invalid="ignore"):
+        t = np.abs(yl) / g_sc[..., None]
     err = np.abs(deq - yl)
     if w.out_dtype == "int8":
         assert (err <= (0.5 + 1.0) * g_sc[..., None]).all()
     elif w.out_dtype == "e2m1":
-        # one step of E2M1 is at most half the value (normal) or 0.5 * s
-        big = t >= 1.0
+        # one step of E2M1 is at most half the value (normal) or 0.5 * s; an
+        # NVFP4 block's largest element may also saturate from up to 6.4 to 6.
+        # An NVFP4 block whose scale rounds to zero (amax * g / 6 <= 2^-10)
+        # dequantizes to zero.
+        zero = np.broadcast_to(g_sc[..., None] == 0, t.shape)
+        if zero.any():
+            assert w.scale_fmt == "e4m3" and (vals[zero] == 0).all()
+            bound0 = 6.0 * 2.0 ** -10 / np.float64(np.float32(w.global_scale))
+            assert (err[zero] <= bound0 * (1 + 2.0 ** -10)).all(), f"{w.name}: zero blocks"
+        # An NVFP4 block scale saturated at 448 leaves t above 6: those codes
+        # saturate too, and the error is what lies beyond 6 * scale.
+        sc_b = np.broadcast_to(g_sc[..., None], t.shape)
+        sat = (t > 6.5) & ~zero
+        if sat.any():
+            assert w.scale_fmt == "e4m3" and (np.abs(vals[sat]) == 6).all()
+            assert (err[sat] <= (t[sat] - 6.0) * sc_b[sat] * (1 + 2.0 ** -10)).all()
+        big = (t >= 1.0) & ~zero & ~sat
+        small = (t < 1.0) & ~zero
         assert (err[big] <= 0.5 * np.abs(yl[big]) + 1e-30).all(), f"{w.name}: dequant error"
-        assert (err[~big] <= np.broadcast_to(g_sc[..., None], t.shape)[~big] * 0.75).all()
+        assert (err[small] <= sc_b[small] * 0.75).all()
     else:
         big = t >= 2.0 ** -6
         assert (err[big] <= rel_tol * np.abs(yl[big])).all(), f"{w.name}: dequant error"

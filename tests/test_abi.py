@@ -79,7 +79,8 @@ def test_enum_values_match_header():
     text = open(HEADER).read()
     for name in ("PQG_OK", "PQG_ERR_INVALID_ARG", "PQG_ERR_UNSUPPORTED", "PQG_ERR_ALIGNMENT",
                  "PQG_ERR_CUDA", "PQG_BF16", "PQG_FP16", "PQG_E4M3", "PQG_INT8", "PQG_E2M1",
-                 "PQG_SCALE_FP32", "PQG_SCALE_UE8M0", "PQG_ROW_MAJOR", "PQG_COL_MAJOR_TMA",
+                 "PQG_SCALE_FP32", "PQG_SCALE_UE8M0", "PQG_SCALE_E4M3", "PQG_ROW_MAJOR",
+                 "PQG_COL_MAJOR_TMA",
                  "PQG_UE8M0_PACKED", "PQG_UE8M0_TILED_128x4"):
         m = re.search(rf"\b{name}\s*=\s*(-?\d+)", text)
         assert m and int(m.group(1)) == getattr(pqg, name), name
@@ -111,6 +112,16 @@ def test_scales_bytes_matches_oracle(E, M, K, G, fmt, layout):
     assert int(np.prod(shape)) * torch.empty((), dtype=dt).element_size() == want
 
 
+@pytest.mark.parametrize("E,M,K", [(1, 4, 256), (1, 8192, 7168), (3, 130, 80), (2, 1, 16)])
+@pytest.mark.parametrize("layout", ["row", "col", "tile128x4"])
+def test_nvfp4_scales_bytes_matches_oracle(E, M, K, layout):
+    import oracle
+    want = oracle.load().pqgo_scales_nbytes(E, M, K, 16, 1, oracle.LAYOUTS[layout])
+    assert pqg.pqg_scales_bytes(E, M, K, 16, pqg.PQG_SCALE_E4M3, pqg.LAYOUTS[layout]) == want
+    shape, dt = pqg.scales_spec(M, K, 16, "e4m3", layout, E)
+    assert int(np.prod(shape)) == want
+
+
 def test_per_token_scales_bytes():
     for K in (80, 7168, 16384):
         assert pqg.pqg_scales_bytes(1, 5, K, K, pqg.PQG_SCALE_FP32, pqg.PQG_ROW_MAJOR) == 5 * 4
@@ -128,6 +139,10 @@ def test_scales_bytes_rejects():
     assert pqg.pqg_scales_bytes(1, 4, 256, 128, S, 9) == pqg.PQG_ERR_INVALID_ARG
     assert pqg.pqg_scales_bytes(1, 4, 256, -128, S, R) == pqg.PQG_ERR_INVALID_ARG
     assert pqg.pqg_scales_bytes(1, 1 << 31, 512, 128, S, R) == pqg.PQG_ERR_INVALID_ARG
+    E4 = pqg.PQG_SCALE_E4M3                          # NVFP4: blocks of 16, byte layouts
+    assert pqg.pqg_scales_bytes(1, 4, 256, 32, E4, R) == pqg.PQG_ERR_UNSUPPORTED
+    assert pqg.pqg_scales_bytes(1, 4, 256, 16, E4, P) == pqg.PQG_ERR_UNSUPPORTED
+    assert pqg.pqg_scales_bytes(1, 4, 200, 16, E4, R) == pqg.PQG_ERR_INVALID_ARG
 
 
 # --------------------------------------------------------------------------
@@ -187,6 +202,41 @@ def test_quant_rejects_before_launch(kw, status):
     before = pqg.pqg_launch_count()
     assert call(**kw) == status
     assert pqg.pqg_launch_count() == before
+
+
+def call_nv(**kw):
+    a = dict(in_ptr=FAKE, out_ptr=FAKE + (1 << 32), scales_ptr=FAKE + (2 << 32),
+             global_scale_ptr=FAKE + (3 << 32), M=4, num_experts=1, K=256,
+             in_dtype=pqg.PQG_BF16, scale_layout=pqg.PQG_ROW_MAJOR, fuse_silu_mul=0,
+             masked_m_ptr=None, expected_m=0, stream=None)
+    a.update(kw)
+    return pqg.pqg_quant_nvfp4(**a)
+
+
+@host_only
+@pytest.mark.parametrize("kw,status", [
+    (dict(global_scale_ptr=0), pqg.PQG_ERR_INVALID_ARG),
+    (dict(global_scale_ptr=FAKE + (3 << 32) + 2), pqg.PQG_ERR_ALIGNMENT),
+    (dict(scale_layout=pqg.PQG_UE8M0_PACKED), pqg.PQG_ERR_UNSUPPORTED),
+    (dict(scale_layout=7), pqg.PQG_ERR_INVALID_ARG),
+    (dict(K=200), pqg.PQG_ERR_INVALID_ARG),
+    (dict(in_dtype=9), pqg.PQG_ERR_INVALID_ARG),
+    (dict(M=-1), pqg.PQG_ERR_INVALID_ARG),
+    (dict(num_experts=4097), pqg.PQG_ERR_INVALID_ARG),
+    (dict(in_ptr=FAKE + 16), pqg.PQG_ERR_ALIGNMENT),
+    (dict(out_ptr=FAKE + (1 << 32) + 8), pqg.PQG_ERR_ALIGNMENT),
+    (dict(out_ptr=FAKE + 256), pqg.PQG_ERR_INVALID_ARG),          # overlaps the input
+])
+def test_nvfp4_rejects_before_launch(kw, status):
+    before = pqg.pqg_launch_count()
+    assert call_nv(**kw) == status
+    assert pqg.pqg_launch_count() == before
+
+
+@host_only
+def test_quant_refers_e4m3_block_scales_to_the_nvfp4_entry():
+    assert call(out_dtype=pqg.PQG_E2M1, scale_fmt=pqg.PQG_SCALE_E4M3,
+                group=16) == pqg.PQG_ERR_UNSUPPORTED
 
 
 @host_only

@@ -45,6 +45,16 @@ MUTANTS = {
     "mxfp4_uses_fmax448": ("ebyte = pqgo_ue8m0_exponent_fmax(amax, out_e2m1 ? PQGO_FMAX_E2M1",
                            "ebyte = pqgo_ue8m0_exponent_fmax(amax, out_e2m1 ? PQGO_FMAX_E4M3"),
     "tile_rows_not_interleaved": ("(r % 32) * 16 + (r / 32) * 4", "(r % 32) * 4 + (r / 32) * 128"),
+    "nvfp4_scale_uses_fmax448": ("float r = (amax / PQGO_FMAX_E2M1) * g;",
+                                 "float r = (amax / PQGO_FMAX_E4M3) * g;"),
+    "nvfp4_global_scale_ignored": ("float r = (amax / PQGO_FMAX_E2M1) * g;",
+                                   "float r = (amax / PQGO_FMAX_E2M1);"),
+    "nvfp4_multiplier_inverted": ("return d == 0.0f ? 0.0f : g / d;",
+                                  "return d == 0.0f ? 0.0f : d / g;"),
+    "nvfp4_zero_scale_unguarded": ("return d == 0.0f ? 0.0f : g / d;", "return g / d;"),
+    "nvfp4_nibbles_swapped": ("qrow[(b * G + i) / 2] = (uint8_t)(lo | (hi << 4));",
+                              "qrow[(b * G + i) / 2] = (uint8_t)(hi | (lo << 4));"),
+    "nvfp4_tile_padding_not_zeroed": ("scales[e * plane + tile128x4_offset(m, b, ng)] = 0;", ";"),
 }
 
 

@@ -220,6 +220,166 @@ def test_mxfp4_dequant_error_bound_and_nibble_order():
     assert (err[t < 1] <= 0.25 * np.broadcast_to(sc, x.shape)[t < 1] + 1e-30).all()
 
 
+# --------------------------------------------------------------------------
+# NVFP4: E2M1 codes in blocks of 16, E4M3 block scales, fp32 global scale g
+# --------------------------------------------------------------------------
+
+E4M3_MIDS = (np.sort(POS_VALS)[1:] + np.sort(POS_VALS)[:-1]) / 2.0
+E2M1_MIDS = (E2M1_MAGS[1:] + E2M1_MAGS[:-1]) / 2.0
+NV_SCALES = (1.0, 2.625, 896.0, 0.37109375, 2.0 ** -12, 5000.0)
+
+
+def _near(v, mids, rel) -> np.ndarray:
+    """|v| within `rel` (relative) of one of the rounding midpoints."""
+    v = np.abs(np.asarray(v, np.float64)).reshape(-1)
+    i = np.clip(np.searchsorted(mids, v), 1, mids.size - 1)
+    d = np.minimum(np.abs(v - mids[i - 1]), np.abs(v - mids[i]))
+    return d <= rel * np.maximum(v, 1e-300)
+
+
+def test_e4m3_decode_matches_torch():
+    got = oracle.e4m3_decode(np.arange(256)).astype(np.float64)
+    lib = torch.arange(256, dtype=torch.int32).to(torch.uint8).view(torch.float8_e4m3fn)
+    lib = lib.double().numpy()
+    assert np.array_equal(np.isnan(got), np.isnan(lib))
+    fin = ~np.isnan(lib)
+    assert np.array_equal(got[fin], lib[fin])
+    assert np.array_equal(np.signbit(got[fin]), np.signbit(lib[fin]))
+
+
+@pytest.mark.parametrize("g", NV_SCALES)
+def test_nvfp4_block_scale_is_nearest_e4m3_of_amax_times_g_over_6(g):
+    """sf = the E4M3 code nearest to amax * g / 6 (exact arithmetic), saturating
+    at 448, except within fp32 rounding of an E4M3 midpoint."""
+    rng = np.random.default_rng(31)
+    a = np.concatenate([log_uniform(rng, 200_000, -34, 17, signed=False),
+                        np.float32([1e-10, 6.0, 3.0, 2688.0])]).astype(np.float32)
+    g32 = np.float32(g)
+    r = a.astype(np.float64) * np.float64(g32) / 6.0
+    near = _near(np.minimum(r, 448.0), E4M3_MIDS, 2.0 ** -21)
+    assert near.mean() < 1e-3
+    got = oracle.nvfp4_block_scale(a, g32)
+    assert np.array_equal(got[~near], brute_e4m3(r)[~near])
+
+
+@pytest.mark.parametrize("g", NV_SCALES)
+def test_nvfp4_multiplier_is_correctly_rounded_g_over_block_scale(g):
+    sf = np.arange(0, 0x7F)
+    m = oracle.nvfp4_multiplier(sf, np.float32(g)).astype(np.float64)
+    assert m[0] == 0.0                                 # a zero block scale zeroes the block
+    exact = np.float64(np.float32(g)) / TABLE[sf[1:]]
+    ulp = np.spacing(np.abs(m[1:]).astype(np.float32)).astype(np.float64)
+    assert (np.abs(m[1:] - exact) <= 0.5 * ulp * (1 + 2.0 ** -20)).all()
+
+
+def _nvfp4_block(w, g, layout="row"):
+    q, s = oracle.quant(w.x, M=w.M, K=w.K, group=16, out_dtype="e2m1", scale_fmt="e4m3",
+                        layout=layout, global_scale=g)
+    x = _f32(w.x).reshape(w.M, -1, 16).astype(np.float64)
+    b = q.reshape(w.M, -1)
+    codes = np.stack([b & 0xF, b >> 4], axis=-1).reshape(w.M, -1, 16)   # element 2i low
+    return x, codes, s
+
+
+@pytest.mark.parametrize("g", (2.625, 0.37109375, 5000.0))
+def test_nvfp4_codes_are_nearest_e2m1_of_x_times_g_over_block_scale(g):
+    """Every code is the E2M1 value nearest to x * g / value(sf) (exact
+    arithmetic, saturating at 6); every block scale is nearest to amax * g / 6;
+    and dequantized values keep within half an E2M1 step."""
+    w = inputs.sweep(M=96, K=1024, seed=33)
+    x = _f32(w.x).reshape(96, -1, 16).astype(np.float64)
+    x[::7, 3] *= 300.0                                 # outlier blocks
+    x[5::11, 9] *= 2.0 ** -40                          # blocks whose scale underflows
+    w = w.with_(x=inputs.bf16_bits(x.astype(np.float32)).reshape(1, 96, 1024))
+    g32 = np.float64(np.float32(g))
+    x, codes, s = _nvfp4_block(w, g)
+    sf = s.reshape(96, -1)
+    amax = np.maximum(np.abs(x).max(-1), np.float64(np.float32(1e-10)))
+    r = amax * g32 / 6.0
+    near_s = _near(np.minimum(r, 448.0), E4M3_MIDS, 2.0 ** -21).reshape(sf.shape)
+    assert np.array_equal(sf[~near_s], brute_e4m3(r)[~near_s.reshape(-1)])
+    d = TABLE[sf][..., None]
+    with np.errstate(divide="ignore", invalid="ignore"):
+        t = x * g32 / d
+        m64 = np.broadcast_to(g32 / d, t.shape)
+    # Codes are pinned except near an E2M1 midpoint, where fp32 rounding of the
+    # multiplier may decide; an exact tie stays pinned (ties to even) when the
+    # multiplier g / value(sf) is exact in fp32.
+    ta_c = np.minimum(np.abs(t), 6.0)
+    near_c = _near(ta_c, E2M1_MIDS, 2.0 ** -21).reshape(t.shape)
+    exact_tie = np.isin(ta_c, E2M1_MIDS) & (m64.astype(np.float32).astype(np.float64) == m64)
+    zero_blk = np.broadcast_to(d == 0, t.shape)
+    assert zero_blk.any()
+    assert np.array_equal(codes[zero_blk], 8 * np.signbit(x[zero_blk]).astype(np.uint8))
+    pinned = (~near_c | exact_tie) & ~zero_blk
+    assert (~pinned).mean() < 5e-3
+    if g == 2.625:                                     # ties do occur: 21/8 over 2^k
+        assert exact_tie.sum() > 20
+    want = brute_e2m1(t).reshape(t.shape)
+    assert np.array_equal(codes[pinned], want[pinned])
+    # dequantization: x ~ code * value(sf) / g; a zero block scale zeroes the block
+    vals = E2M1_MAGS[codes & 7] * np.where(codes & 8, -1.0, 1.0)
+    err = np.abs(vals * d / g32 - x)
+    s_x = np.broadcast_to(d / g32, x.shape)
+    zero = np.broadcast_to(d == 0, x.shape)
+    assert (vals[zero] == 0).all()
+    assert (np.abs(x[zero]) <= 6.0 * 2.0 ** -10 / g32).all()
+    ta = np.where(zero, 0.0, np.abs(t))
+    big, small, sat = (ta >= 1) & (ta <= 6), (ta < 1) & ~zero, ta > 6
+    assert (err[big] <= 0.25 * np.abs(x[big]) * (1 + 2.0 ** -20)).all()
+    assert (err[small] <= 0.25 * s_x[small] * (1 + 2.0 ** -20)).all()
+    assert (err[sat] <= (ta[sat] - 6.0) * s_x[sat] * (1 + 2.0 ** -20)).all()
+    if g < 448 * 6 / 300.0 / 8:                        # no block scale saturated
+        assert (ta <= 6.0 * (1 + 2.0 ** -4) * (1 + 2.0 ** -20)).all()
+
+
+def test_nvfp4_zero_block_scale_gives_signed_zero_codes():
+    v = np.zeros(48, np.float32)
+    v[5] = -0.0                                        # block 0: all zero (amax floored)
+    v[16:19] = [2.0 ** -100, -(2.0 ** -100), -(2.0 ** -120)]   # block 1: underflows
+    v[32] = 1.0                                        # block 2: ordinary
+    w = inputs.Workload("zeros", inputs.bf16_bits(v).reshape(1, 1, 48), M=1, K=48, group=16)
+    x, codes, s = _nvfp4_block(w, 1.0)
+    assert s.reshape(-1).tolist()[:2] == [0, 0]
+    assert codes[0, 0].tolist() == [8 if i == 5 else 0 for i in range(16)]
+    assert codes[0, 1, :3].tolist() == [0, 8, 8] and (codes[0, 1, 3:] == 0).all()
+    assert s.reshape(-1)[2] == brute_e4m3([1.0 / 6.0])[0]
+
+
+def test_nvfp4_layouts_and_masking():
+    """row, col and 128x4-tiled NVFP4 scales hold the same bytes at their
+    positions; masked rows stay untouched; full masks equal flat calls."""
+    M, K = 130, 5 * 16                                 # ng = 5: ragged tiles
+    x = inputs.bf16_bits(inputs.normal((1, M, K), 34) * 2)
+    q_r, s_r = oracle.quant(x, M=M, K=K, group=16, out_dtype="e2m1", scale_fmt="e4m3",
+                            layout="row", global_scale=2.625)
+    q_c, s_c = oracle.quant(x, M=M, K=K, group=16, out_dtype="e2m1", scale_fmt="e4m3",
+                            layout="col", global_scale=2.625)
+    q_t, s_t = oracle.quant(x, M=M, K=K, group=16, out_dtype="e2m1", scale_fmt="e4m3",
+                            layout="tile128x4", global_scale=2.625)
+    assert np.array_equal(q_r, q_c) and np.array_equal(q_r, q_t)
+    row = s_r.reshape(M, 5)
+    assert np.array_equal(s_c.reshape(5, 132)[:, :M], row.T)
+    til = s_t.reshape(-1)
+    for (m, g), byte in {(0, 0): 0, (1, 0): 16, (33, 1): 21, (127, 3): 511, (0, 4): 512,
+                         (129, 4): 1552}.items():
+        assert int(til[byte]) == int(row[m, g]), (m, g, byte)
+    for g in (5, 6, 7):                                # padding columns of row 129
+        assert til[1024 + 1 * 16 + 512 + g % 4] == 0
+    E = 3
+    xe = inputs.bf16_bits(inputs.normal((E, 8, 2 * 64), 35))
+    mm = np.array([0, 5, 8], np.int32)
+    q, s = oracle.quant(xe, E=E, M=8, K=64, group=16, out_dtype="e2m1", scale_fmt="e4m3",
+                        layout="row", fused=True, masked_m=mm, global_scale=2.625)
+    q, s = q.reshape(E, 8, 32), s.reshape(E, 8, 4)
+    for e in range(E):
+        assert (q[e, mm[e]:] == 0xA5).all() and (s[e, mm[e]:] == 0xA5).all()
+        qf, sf = oracle.quant(xe[e], M=8, K=64, group=16, out_dtype="e2m1", scale_fmt="e4m3",
+                              layout="row", fused=True, global_scale=2.625)
+        assert np.array_equal(q[e, :mm[e]], qf.reshape(8, 32)[:mm[e]])
+        assert np.array_equal(s[e, :mm[e]], sf.reshape(8, 4)[:mm[e]])
+
+
 def test_int8_encoder_matches_numpy_rint():
     rng = np.random.default_rng(13)
     t = np.concatenate([rng.uniform(-200, 200, 500_000).astype(np.float32),
@@ -283,6 +443,17 @@ def _golden_group(entry) -> np.ndarray:
 
 @pytest.mark.parametrize("entry", json.load(open(GOLDEN))["groups"], ids=lambda e: e["name"])
 def test_worked_group(entry):
+    if "nvfp4" in entry:
+        v = np.zeros(entry["K"], np.float32)
+        for i, x in entry["values"].items():
+            v[int(i)] = x
+        nv = entry["nvfp4"]
+        q, s = oracle.quant(inputs.bf16_bits(v), M=1, K=entry["K"], group=16, out_dtype="e2m1",
+                            scale_fmt="e4m3", layout="row", global_scale=nv["global_scale"])
+        assert s.reshape(-1).tolist() == nv["scales"]
+        for i, b in nv["bytes"].items():
+            assert int(q.reshape(-1)[int(i)]) == b, (entry["name"], i)
+        return
     if "e2m1" in entry:
         v = np.zeros(entry["group"], np.float32)
         for i, x in entry["values"].items():
@@ -531,6 +702,14 @@ def test_oracle_rejects_unsupported_combinations():
         oracle.quant(x, M=4, K=256, group=128, out_dtype="int8", scale_fmt="ue8m0")
     with pytest.raises(ValueError):
         oracle.quant(x, M=4, K=256, group=128, scale_fmt="fp32", layout="packed")
+    with pytest.raises(ValueError):                       # NVFP4 needs a global scale
+        oracle.quant(x, M=4, K=256, group=16, out_dtype="e2m1", scale_fmt="e4m3")
+    with pytest.raises(ValueError):
+        oracle.quant(x, M=4, K=256, group=16, out_dtype="e2m1", scale_fmt="e4m3",
+                     layout="packed", global_scale=1.0)
+    with pytest.raises(ValueError):
+        oracle.quant(x, M=4, K=256, group=16, out_dtype="e2m1", scale_fmt="e4m3",
+                     global_scale=-1.0)
     nan = np.full((1, 4, 256), 0x7FC0, np.uint16)
     with pytest.raises(ValueError):
         oracle.quant(nan, M=4, K=256, group=128)

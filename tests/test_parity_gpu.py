@@ -385,3 +385,82 @@ def test_mxfp4_every_input_value(in_dtype, carrier):
 
 def test_mxfp4_full_size():
     check_exact(inputs.mxfp4())
+
+
+# --------------------------------------------------------------------------
+# NVFP4: E2M1 codes in blocks of 16, E4M3 block scales, fp32 global scale
+# --------------------------------------------------------------------------
+
+NV_LAYOUTS = ["row", "col", "tile128x4"]
+
+
+def make_nv(M, K, g, layout, in_dtype="bf16", fused=False, E=1, seed=0, masked_m=None,
+            expected_m=0):
+    w = make(M, K, 16, ("e2m1", "e4m3", layout), in_dtype, fused=fused, E=E, seed=seed,
+             masked_m=masked_m, expected_m=expected_m)
+    return w.with_(name=f"{w.name}_g{g}", global_scale=g)
+
+
+@pytest.mark.parametrize("layout", NV_LAYOUTS)
+@pytest.mark.parametrize("in_dtype", ["bf16", "fp16"])
+@pytest.mark.parametrize("g", [1.0, 2.625, 0.37109375, 5000.0, 2.0 ** -12])
+def test_nvfp4_bit_exact(layout, in_dtype, g):
+    for M, K in [(37, 640), (5, 16), (3, 48), (130, 2048), (1, 7168), (2, 8208)]:
+        check_exact(make_nv(M, K, g, layout, in_dtype, seed=M + K + 11))
+
+
+@pytest.mark.parametrize("in_dtype", ["bf16", "fp16"])
+@pytest.mark.parametrize("carrier,g", [(6.0, 1.0), (1.0, 1.0), (1000.0, 2.625), (3.0, 896.0)])
+def test_nvfp4_every_input_value(in_dtype, carrier, g):
+    """Every finite input value, alone with a carrier in its block (and negated
+    in the next block), through the block scale and the codes."""
+    import oracle
+    bits = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    vals = oracle.decode(bits, in_dtype)
+    bits = bits[np.isfinite(vals)]
+    n = bits.size
+    cb = inputs.to_bits(np.float32([carrier]), in_dtype)[0]
+    x = np.full((1, n, 32), cb, np.uint16)
+    x[0, :, 0] = bits
+    x[0, :, 17] = bits ^ 0x8000
+    check_exact(inputs.Workload("exhaustive_nvfp4", x, M=n, K=32, group=16, in_dtype=in_dtype,
+                                out_dtype="e2m1", scale_fmt="e4m3", layout="row",
+                                global_scale=g))
+
+
+@pytest.mark.parametrize("layout", ["row", "tile128x4"])
+def test_nvfp4_fused_and_masked(layout):
+    E, M, K = 5, 37, 640
+    mm = np.array([0, 37, 1, 99, -3], np.int32)
+    check_exact(make_nv(M, K, 2.625, layout, E=E, seed=61, masked_m=mm, expected_m=8))
+    check_fused(make_nv(M, K, 2.625, layout, fused=True, E=E, seed=62, masked_m=mm,
+                        expected_m=8), max_flip_frac=1e-3)
+    check_fused(make_nv(130, 2048, 1.0, layout, fused=True, seed=63), max_flip_frac=1e-3)
+    check_exact(make_nv(M, K, 2.625, layout, E=40, seed=64,
+                        masked_m=np.arange(40, dtype=np.int32) % (M + 1)))
+
+
+def test_nvfp4_global_scale_written_by_the_preceding_kernel():
+    """The kernel reads g on the device after the stream's previous work: a
+    fill issued just before the call decides the result."""
+    w = make_nv(130, 2048, 2.625, "tile128x4", seed=65)
+    x = torch.from_numpy(np.ascontiguousarray(w.x).view(np.int16)).view(torch.bfloat16).cuda()
+    out, sc = pqg.allocate_outputs(w.M, w.K, 16, out_dtype="e2m1", scale_fmt="e4m3",
+                                   layout="tile128x4", device="cuda")
+    out.fill_(SENTINEL)                      # padding rows must stay as the oracle leaves them
+    sc.fill_(SENTINEL)
+    gsc = torch.ones(1, dtype=torch.float32, device="cuda")
+    torch.cuda.synchronize()
+    for _ in range(3):
+        gsc.fill_(1.0)
+        gsc.fill_(2.625)
+        pqg.quant(x, out, sc, group=16, out_dtype="e2m1", scale_fmt="e4m3", layout="tile128x4",
+                  global_scale=gsc)
+    torch.cuda.synchronize()
+    rq, rs = run_oracle(w)
+    assert_same(out.cpu().numpy().reshape(-1), rq, "codes")
+    assert_same(sc.cpu().numpy().reshape(-1), rs, "scales")
+
+
+def test_nvfp4_full_size():
+    check_exact(inputs.nvfp4())

@@ -48,7 +48,8 @@ def workloads():
     from precision_activation_quantization_b200 import inputs
     return {
         "flat_hidden": lambda: inputs.flat_hidden(),
-        "flat_hidden_fp32": lambda: inputs.flat_hidden(layout="row", scale_fmt="fp32"),
+        "flat_hidden_fp32": lambda: inputs.flat_hidden(layout="row", scale_fmt="fp32").with_(
+            name="flat_8192x7168_fp32_row"),
         "per_token": lambda: inputs.flat_hidden(layout="row", scale_fmt="fp32").with_(
             group=7168, name="per_token_8192x7168"),
         "mxfp4": lambda: inputs.mxfp4(),

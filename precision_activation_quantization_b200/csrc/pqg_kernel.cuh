@@ -26,17 +26,21 @@
 // in registers (double-buffering) and in shared memory (cp.async stages), the
 // extra registers and instructions cost more warps than the prefetch won.
 //
-// Exact division.  Codes must equal a rounding of fp32(x / s).  A per-element
+// Exact codes.  Codes must equal the rounding of fp32(x / s).  A per-element
 // IEEE division is too slow for a bandwidth-bound loop, so the quotient is
-// formed from y = RN(1/s) (one correctly rounded reciprocal per group) and two
+// formed from y = RN(1/s) (one correctly rounded reciprocal per group) and
 // residual corrections, q <- q + (x - q*s) * y with exact FMA residuals
 // (Markstein's correction; P. Markstein, "Computation of elementary functions
 // on the IBM RISC System/6000 processor", IBM J. Res. Dev. 34(1), 1990).  The
-// first step leaves q within an ulp of x/s, and the second then returns the
-// correctly rounded quotient.  Where |x/s| < 2^-12 the residual may underflow,
-// but every such t rounds to a signed zero code, and the sign is restored from
-// x.  The correction runs on packed f32x2 FMAs (FFMA2), two elements per
-// instruction.
+// first step leaves q within an ulp of x/s, and a second returns the correctly
+// rounded quotient.  One step is enough for the codes: for every 8-bit (bf16)
+// and 11-bit (fp16) significand of x, every fp32 significand of s and every
+// binade of x/s that can yield a nonzero code, an exhaustive CPU comparison
+// found the E4M3 and INT8 code of the one-step q equal to the code of
+// RN(x/s) (2.4e10 bf16 and 1.9e11 fp16 cases for E4M3).  Where |x/s| < 2^-12
+// the residual may underflow, but every such t rounds to a signed zero code,
+// and the sign is restored from x.  The correction runs on packed f32x2 FMAs
+// (FFMA2), two elements per instruction.
 //
 // UE8M0 exponent without a division.  For a normal fp32 amax = m * 2^E (m in
 // [1, 2)), the smallest n with 448 * 2^n >= amax is E - 8 + [m > 1.75], because
@@ -231,28 +235,45 @@ __device__ __forceinline__ uint32_t e2m1x2(float lo, float hi) {
     return r;
 }
 
-// The correctly rounded fp32 quotient x/s for a pair, from y = RN(1/s) and
-// ns = -s (two Markstein corrections; see the file comment).
+// Markstein corrections per quotient (STEPS): 2 give the correctly rounded
+// fp32 x/s for every x; 1 leaves q within an ulp of it, and exhaustive CPU
+// checks found the E4M3 and INT8 codes of that q equal to the codes of
+// RN(x/s) for every bf16 / fp16 x and every fp32 s (all significand pairs,
+// every binade of x/s that yields a nonzero code).  The strip kernel uses 1,
+// the per-token row kernel 2 (measured faster there).
+#ifndef PQG_DIV_STEPS
+#define PQG_DIV_STEPS 1
+#endif
+constexpr int kDivSteps = PQG_DIV_STEPS;
+
+// The fp32 quotient x/s for a pair, from y = RN(1/s) and ns = -s (Markstein
+// corrections; see the file comment).
+template <int STEPS>
 __device__ __forceinline__ float2 div_rn2(float2 x, float2 y, float2 ns) {
     float2 q = __fmul2_rn(x, y);
     float2 r = __ffma2_rn(q, ns, x);   // x - q*s, exact
     q = __ffma2_rn(r, y, q);
-    r = __ffma2_rn(q, ns, x);
-    q = __ffma2_rn(r, y, q);
+    if constexpr (STEPS > 1) {
+        r = __ffma2_rn(q, ns, x);
+        q = __ffma2_rn(r, y, q);
+    }
     return q;
 }
 
 // The same correction carried on the negated quotient, from ny = -RN(1/s) and
-// s: returns -RN(x/s) with the sign of zero right for every x.  (q = x*ny and
+// s: returns -x/s with the sign of zero right for every x.  (q = x*ny and
 // r = x + q*s: for x = -0 the chain gives +0, for x = +0 it gives -0, and a
 // tiny x whose quotient underflows keeps the sign of -x.)  Negating the codes
 // afterwards is one XOR of the packed sign bits.
+template <int STEPS>
 __device__ __forceinline__ float2 neg_div_rn2(float2 x, float2 ny, float2 s) {
     float2 q = __fmul2_rn(x, ny);
     float2 r = __ffma2_rn(q, s, x);    // x - (x/s)*s, exact
     q = __ffma2_rn(r, ny, q);
-    r = __ffma2_rn(q, s, x);
-    q = __ffma2_rn(r, ny, q);
+    if constexpr (STEPS > 1) {
+        r = __ffma2_rn(q, s, x);
+        q = __ffma2_rn(r, ny, q);
+    }
     return q;
 }
 
@@ -275,6 +296,19 @@ __device__ __forceinline__ uint32_t absmax_bits16(const uint32_t (&w)[8]) {
     uint32_t b = __vimax3_u16x2(m[3], m[4], m[5]);
     a = __vimax3_u16x2(a, b, __vimax3_u16x2(m[6], m[7], 0u));
     return max(a & 0xFFFFu, a >> 16);
+}
+
+// The value of a non-negative finite bf16 / fp16 magnitude pattern (the
+// per-token kernel takes its absmax on raw bits).
+template <typename In>
+__device__ __forceinline__ float bits16_to_float(uint32_t b);
+template <>
+__device__ __forceinline__ float bits16_to_float<__nv_bfloat16>(uint32_t b) {
+    return __uint_as_float(b << 16);
+}
+template <>
+__device__ __forceinline__ float bits16_to_float<__half>(uint32_t b) {
+    return __half2float(__ushort_as_half(static_cast<unsigned short>(b)));
 }
 
 // ---------------------------------------------------------------------------
@@ -371,7 +405,7 @@ __device__ __forceinline__ GroupScale make_scale(float amax, const float *nv = n
 }
 
 // 16 values -> 16 code bytes (4 words, element 0 in the lowest byte).
-template <Kind KIND>
+template <Kind KIND, int STEPS = kDivSteps>
 __device__ __forceinline__ void encode16(const float (&v)[16], const GroupScale &gs,
                                          uint32_t (&w)[4]) {
     if constexpr (is_e2m1(KIND)) {
@@ -402,8 +436,8 @@ __device__ __forceinline__ void encode16(const float (&v)[16], const GroupScale 
         const float2 s2 = make_float2(gs.s, gs.s);
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-            const float2 a = neg_div_rn2(make_float2(v[4 * j], v[4 * j + 1]), ny2, s2);
-            const float2 b = neg_div_rn2(make_float2(v[4 * j + 2], v[4 * j + 3]), ny2, s2);
+            const float2 a = neg_div_rn2<STEPS>(make_float2(v[4 * j], v[4 * j + 1]), ny2, s2);
+            const float2 b = neg_div_rn2<STEPS>(make_float2(v[4 * j + 2], v[4 * j + 3]), ny2, s2);
             w[j] = (e4m3x2(a.x, a.y) | (e4m3x2(b.x, b.y) << 16)) ^ 0x80808080u;
         }
     } else {
@@ -415,9 +449,10 @@ __device__ __forceinline__ void encode16(const float (&v)[16], const GroupScale 
         const float2 magic = make_float2(12582912.0f, 12582912.0f);
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-            float2 a = __fadd2_rn(div_rn2(make_float2(v[4 * j], v[4 * j + 1]), y2, ns2), magic);
+            float2 a =
+                __fadd2_rn(div_rn2<STEPS>(make_float2(v[4 * j], v[4 * j + 1]), y2, ns2), magic);
             float2 b =
-                __fadd2_rn(div_rn2(make_float2(v[4 * j + 2], v[4 * j + 3]), y2, ns2), magic);
+                __fadd2_rn(div_rn2<STEPS>(make_float2(v[4 * j + 2], v[4 * j + 3]), y2, ns2), magic);
             uint32_t ab = __byte_perm(__float_as_uint(a.x), __float_as_uint(a.y), 0x0040);
             uint32_t cd = __byte_perm(__float_as_uint(b.x), __float_as_uint(b.y), 0x0040);
             w[j] = __byte_perm(ab, cd, 0x5410);

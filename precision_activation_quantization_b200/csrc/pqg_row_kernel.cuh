@@ -22,6 +22,11 @@ namespace pqg {
 
 constexpr int kRowThreads = 256;  // 8 warps per CTA
 
+// Markstein corrections per code of the row kernel (see div_rn2).
+#ifndef PQG_ROW_DIV_STEPS
+#define PQG_ROW_DIV_STEPS 2
+#endif
+
 template <typename In, Kind KIND, bool FUSED, int SLOTS>
 __global__ void __launch_bounds__(kRowThreads)
     row_quant_kernel(const __grid_constant__ Params p) {
@@ -70,24 +75,31 @@ __global__ void __launch_bounds__(kRowThreads)
                 }
             }
         }
-        float v[SLOTS][16];
+        // Fused rows keep silu(gate) * up in registers; plain rows keep the raw
+        // 16-bit values (half the registers) and take the absmax on their
+        // magnitude bits, widening only to quantize.
+        float v[FUSED ? SLOTS : 1][16];
         float amax = 0.0f;
+        if constexpr (FUSED) {
 #pragma unroll
-        for (int j = 0; j < SLOTS; ++j) {
+            for (int j = 0; j < SLOTS; ++j) {
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                widen2<In>(x[j][i], v[j][2 * i], v[j][2 * i + 1]);
-                if constexpr (FUSED) {
-                    float u0, u1;
+                for (int i = 0; i < 8; ++i) {
+                    float g0, g1, u0, u1;
+                    widen2<In>(x[j][i], g0, g1);
                     widen2<In>(u[j][i], u0, u1);
-                    const float2 y =
-                        silu_mul2(make_float2(v[j][2 * i], v[j][2 * i + 1]), make_float2(u0, u1));
+                    const float2 y = silu_mul2(make_float2(g0, g1), make_float2(u0, u1));
                     v[j][2 * i] = y.x;
                     v[j][2 * i + 1] = y.y;
                 }
-            }
 #pragma unroll
-            for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[j][i]));
+                for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[j][i]));
+            }
+        } else {
+            uint32_t ab = 0;
+#pragma unroll
+            for (int j = 0; j < SLOTS; ++j) ab = max(ab, absmax_bits16(x[j]));
+            amax = bits16_to_float<In>(ab);
         }
 
         // -- row absmax: warp, then across the row's warps ---------------------
@@ -108,7 +120,14 @@ __global__ void __launch_bounds__(kRowThreads)
                 const uint32_t slot = tid + j * tpr;
                 if (slot < nslots) {
                     uint32_t w[4];
-                    encode16<KIND>(v[j], gs, w);
+                    if constexpr (FUSED) {
+                        encode16<KIND, PQG_ROW_DIV_STEPS>(v[j], gs, w);
+                    } else {
+                        float vj[16];
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) widen2<In>(x[j][i], vj[2 * i], vj[2 * i + 1]);
+                        encode16<KIND, PQG_ROW_DIV_STEPS>(vj, gs, w);
+                    }
                     store16B(dst + slot * 16u, w[0], w[1], w[2], w[3]);
                 }
             }

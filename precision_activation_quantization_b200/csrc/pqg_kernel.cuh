@@ -235,6 +235,49 @@ __device__ __forceinline__ uint32_t e2m1x2(float lo, float hi) {
     return r;
 }
 
+// FP4 code bytes packed by a vector move (1) or by shifts (0).
+#ifndef PQG_E2M1_VECPACK
+#define PQG_E2M1_VECPACK 1
+#endif
+// E4M3 code pairs packed by a vector move (1) or by shift/or (0).
+#ifndef PQG_E4M3_VECPACK
+#define PQG_E4M3_VECPACK 1
+#endif
+
+// Four E4M3 codes as one word, (a0, a1) in the low half: two conversions and
+// a vector move.
+__device__ __forceinline__ uint32_t e4m3x4(float a0, float a1, float b0, float b1) {
+#if PQG_E4M3_VECPACK
+    uint32_t r;
+    asm("{\n\t.reg .b16 p, q;\n\t"
+        "cvt.rn.satfinite.e4m3x2.f32 p, %2, %1;\n\t"
+        "cvt.rn.satfinite.e4m3x2.f32 q, %4, %3;\n\t"
+        "mov.b32 %0, {p, q};\n\t}"
+        : "=r"(r)
+        : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+    return r;
+#else
+    return e4m3x2(a0, a1) | (e4m3x2(b0, b1) << 16);
+#endif
+}
+
+// Eight E2M1 codes (four pairs, pair k from (v[2k], v[2k+1])) as one word:
+// the four code bytes are packed by a vector move, so the assembler is free to
+// place each conversion's byte.
+__device__ __forceinline__ uint32_t e2m1x8(float a0, float a1, float b0, float b1, float c0,
+                                           float c1, float d0, float d1) {
+    uint32_t r;
+    asm("{\n\t.reg .b8 p, q, s, t;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 p, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 q, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 s, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 t, %8, %7;\n\t"
+        "mov.b32 %0, {p, q, s, t};\n\t}"
+        : "=r"(r)
+        : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1), "f"(d0), "f"(d1));
+    return r;
+}
+
 // Markstein corrections per quotient (STEPS): 2 give the correctly rounded
 // fp32 x/s for every x; 1 leaves q within an ulp of it, and exhaustive CPU
 // checks found the E4M3 and INT8 codes of that q equal to the codes of
@@ -413,6 +456,13 @@ __device__ __forceinline__ void encode16(const float (&v)[16], const GroupScale 
         const float2 m2 = make_float2(gs.mult, gs.mult);
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
+#if PQG_E2M1_VECPACK
+            float2 t[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                t[k] = __fmul2_rn(make_float2(v[8 * j + 2 * k], v[8 * j + 2 * k + 1]), m2);
+            w[j] = e2m1x8(t[0].x, t[0].y, t[1].x, t[1].y, t[2].x, t[2].y, t[3].x, t[3].y);
+#else
             uint32_t word = 0;
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
@@ -420,6 +470,7 @@ __device__ __forceinline__ void encode16(const float (&v)[16], const GroupScale 
                 word |= e2m1x2(t.x, t.y) << (8 * k);
             }
             w[j] = word;
+#endif
         }
     } else if constexpr (KIND == Kind::E4M3_UE8M0) {
         const float2 m2 = make_float2(gs.mult, gs.mult);
@@ -428,7 +479,7 @@ __device__ __forceinline__ void encode16(const float (&v)[16], const GroupScale 
             // multiplying by a power of two is exact: t = x / s
             float2 a = __fmul2_rn(make_float2(v[4 * j], v[4 * j + 1]), m2);
             float2 b = __fmul2_rn(make_float2(v[4 * j + 2], v[4 * j + 3]), m2);
-            w[j] = e4m3x2(a.x, a.y) | (e4m3x2(b.x, b.y) << 16);
+            w[j] = e4m3x4(a.x, a.y, b.x, b.y);
         }
     } else if constexpr (KIND == Kind::E4M3_FP32) {
         // codes of -t, then the four sign bits flipped at once
@@ -438,7 +489,7 @@ __device__ __forceinline__ void encode16(const float (&v)[16], const GroupScale 
         for (int j = 0; j < 4; ++j) {
             const float2 a = neg_div_rn2<STEPS>(make_float2(v[4 * j], v[4 * j + 1]), ny2, s2);
             const float2 b = neg_div_rn2<STEPS>(make_float2(v[4 * j + 2], v[4 * j + 3]), ny2, s2);
-            w[j] = (e4m3x2(a.x, a.y) | (e4m3x2(b.x, b.y) << 16)) ^ 0x80808080u;
+            w[j] = e4m3x4(a.x, a.y, b.x, b.y) ^ 0x80808080u;
         }
     } else {
         // INT8: adding 1.5 * 2^23 rounds |t| < 2^22 to an integer (ties to even)
@@ -670,6 +721,16 @@ __device__ __forceinline__ void quantize_strip(const uint32_t (&x)[8], const uin
         gs.e8 = KIND == Kind::E2M1_UE8M0 ? ue8m0_exponent_e2m1(amax) : ue8m0_exponent(amax);
         const uint16_t p2 = static_cast<uint16_t>((254u - gs.e8) << 7);  // bf16 2^(127-e)
         if constexpr (KIND == Kind::E2M1_UE8M0) {
+#if PQG_E2M1_VECPACK
+            float t[16];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                t[2 * i] = mul_bf16_pow2(static_cast<uint16_t>(x[i] & 0xFFFFu), p2);
+                t[2 * i + 1] = mul_bf16_pow2(static_cast<uint16_t>(x[i] >> 16), p2);
+            }
+            w[0] = e2m1x8(t[0], t[1], t[2], t[3], t[4], t[5], t[6], t[7]);
+            w[1] = e2m1x8(t[8], t[9], t[10], t[11], t[12], t[13], t[14], t[15]);
+#else
             w[0] = w[1] = 0u;
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
@@ -677,6 +738,7 @@ __device__ __forceinline__ void quantize_strip(const uint32_t (&x)[8], const uin
                 const float t1 = mul_bf16_pow2(static_cast<uint16_t>(x[i] >> 16), p2);
                 w[i >> 2] |= e2m1x2(t0, t1) << (8 * (i & 3));
             }
+#endif
         } else {
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
@@ -685,7 +747,7 @@ __device__ __forceinline__ void quantize_strip(const uint32_t (&x)[8], const uin
                 const float t1 = mul_bf16_pow2(static_cast<uint16_t>(a >> 16), p2);
                 const float t2 = mul_bf16_pow2(static_cast<uint16_t>(b & 0xFFFFu), p2);
                 const float t3 = mul_bf16_pow2(static_cast<uint16_t>(b >> 16), p2);
-                w[j] = e4m3x2(t0, t1) | (e4m3x2(t2, t3) << 16);
+                w[j] = e4m3x4(t0, t1, t2, t3);
             }
         }
     } else {

@@ -134,7 +134,8 @@ enum pqg_scale_layout {
  *          [num_experts][M][K/2] bytes of E2M1 code pairs.  16-byte aligned.
  * scales   device.  pqg_scales_bytes(num_experts, M, K, group, scale_fmt,
  *          scale_layout) bytes in the chosen layout.  4-byte aligned for fp32
- *          scales and packed words, any alignment for UE8M0 bytes.
+ *          scales, packed words and the 128x4 tiled layout; any alignment for
+ *          row- or column-major UE8M0 bytes.
  * M        rows per expert (with masked_m: the capacity M_max of each expert).
  *          M >= 0; M == 0 launches nothing.
  * num_experts  1 ..= 4096.  With masked_m == NULL every expert's M rows

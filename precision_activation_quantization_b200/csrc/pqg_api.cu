@@ -117,8 +117,9 @@ int quant_impl(const void *in, void *out, void *scales, const float *global_scal
     if (nvfp4 && global_scale == nullptr) return PQG_ERR_INVALID_ARG;
     if (!aligned(in, 32) || !aligned(out, 16)) return PQG_ERR_ALIGNMENT;
     if (nvfp4 && !aligned(global_scale, 4)) return PQG_ERR_ALIGNMENT;
-    if (scale_fmt == PQG_SCALE_FP32 || scale_layout == PQG_UE8M0_PACKED) {
-        if (!aligned(scales, 4)) return PQG_ERR_ALIGNMENT;
+    if (scale_fmt == PQG_SCALE_FP32 || scale_layout == PQG_UE8M0_PACKED ||
+        scale_layout == PQG_UE8M0_TILED_128x4) {
+        if (!aligned(scales, 4)) return PQG_ERR_ALIGNMENT;  // word stores
     }
     if (masked_m != nullptr && !aligned(masked_m, 4)) return PQG_ERR_ALIGNMENT;
 

@@ -693,6 +693,12 @@ __device__ __forceinline__ void load_chunk(Chunk<ITEMS, FUSED> &ch, uint32_t s, 
     }
 }
 
+// UE8M0 exponents of the 128x4 tiled layout stored as one word per 4 groups
+// (1; the scale buffer is then 4-byte aligned) or byte by byte (0).
+#ifndef PQG_TILED_WORDS
+#define PQG_TILED_WORDS 1
+#endif
+
 // bf16 UE8M0 through the mixed-precision FMA path (1) or by widening (0).
 #ifndef PQG_UE8M0_MIXED
 #define PQG_UE8M0_MIXED 1
@@ -794,7 +800,19 @@ __device__ __forceinline__ void quantize_strip(const uint32_t (&x)[8], const uin
                 reinterpret_cast<uint32_t *>(sc)[static_cast<uint64_t>(g >> 2) * p.mpad + row] =
                     packed_word;
         } else if (p.layout == kTiled128x4) {
+#if PQG_TILED_WORDS
+            if constexpr (is_ue8m0(KIND)) {
+                // groups 4j..4j+3 of the row are 4 consecutive bytes of one tile:
+                // one word, its padding bytes already 0
+                if ((g & 3u) == 0u)
+                    *reinterpret_cast<uint32_t *>(sc + tile128x4_offset(row, g, p.ng)) =
+                        packed_word;
+            } else {
+                store_tiled(sc, row, g, p.ng, gs.e8);
+            }
+#else
             store_tiled(sc, row, g, p.ng, gs.e8);
+#endif
         } else {
             const uint64_t idx = (p.layout == kRowMajor) ? static_cast<uint64_t>(row) * p.ng + g
                                                          : static_cast<uint64_t>(g) * p.mpad + row;

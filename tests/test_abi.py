@@ -192,6 +192,8 @@ def call(**kw):
     (dict(scales_ptr=FAKE + (2 << 32) + 2), pqg.PQG_ERR_ALIGNMENT),
     (dict(scales_ptr=FAKE + (2 << 32) + 2, scale_fmt=pqg.PQG_SCALE_UE8M0,
           scale_layout=pqg.PQG_UE8M0_PACKED), pqg.PQG_ERR_ALIGNMENT),
+    (dict(scales_ptr=FAKE + (2 << 32) + 1, scale_fmt=pqg.PQG_SCALE_UE8M0,
+          scale_layout=pqg.PQG_UE8M0_TILED_128x4), pqg.PQG_ERR_ALIGNMENT),   # word stores
     (dict(masked_m_ptr=FAKE + (3 << 32) + 2), pqg.PQG_ERR_ALIGNMENT),
     (dict(out_ptr=FAKE + 512), pqg.PQG_ERR_INVALID_ARG),          # overlaps the input
     (dict(scales_ptr=FAKE + (1 << 32) + 64), pqg.PQG_ERR_INVALID_ARG),  # overlaps out

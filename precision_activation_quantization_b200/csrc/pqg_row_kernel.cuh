@@ -27,6 +27,23 @@ constexpr int kRowThreads = 256;  // 8 warps per CTA
 #define PQG_ROW_DIV_STEPS 2
 #endif
 
+// The scale of row `row` of expert e.  One group per row: row-major,
+// column-major and packed all put it at element / word `row` of the expert's
+// plane; the tiled layout has one tile column.
+template <Kind KIND>
+__device__ __forceinline__ void store_row_scale(const Params &p, uint32_t e, uint32_t row,
+                                                const GroupScale &gs) {
+    uint8_t *sc = p.scales + e * p.scale_expert_bytes;
+    if (p.layout == kPacked)
+        reinterpret_cast<uint32_t *>(sc)[row] = gs.e8;  // bytes 1..3 are 0
+    else if (p.layout == kTiled128x4)
+        store_tiled(sc, row, 0u, 1u, gs.e8);
+    else if constexpr (is_ue8m0(KIND))
+        sc[row] = static_cast<uint8_t>(gs.e8);
+    else
+        reinterpret_cast<float *>(sc)[row] = gs.s;
+}
+
 template <typename In, Kind KIND, bool FUSED, int SLOTS>
 __global__ void __launch_bounds__(kRowThreads)
     row_quant_kernel(const __grid_constant__ Params p) {
@@ -131,20 +148,7 @@ __global__ void __launch_bounds__(kRowThreads)
                     store16B(dst + slot * 16u, w[0], w[1], w[2], w[3]);
                 }
             }
-            if (tid == 0) {
-                // one group per row: row-major, column-major and packed all put
-                // row r's scale at element / word r of the expert's plane; the
-                // tiled layout has one tile column
-                uint8_t *sc = p.scales + sp.e * p.scale_expert_bytes;
-                if (p.layout == kPacked)
-                    reinterpret_cast<uint32_t *>(sc)[row] = gs.e8;  // bytes 1..3 are 0
-                else if (p.layout == kTiled128x4)
-                    store_tiled(sc, row, 0u, 1u, gs.e8);
-                else if constexpr (is_ue8m0(KIND))
-                    sc[row] = static_cast<uint8_t>(gs.e8);
-                else
-                    reinterpret_cast<float *>(sc)[row] = gs.s;
-            }
+            if (tid == 0) store_row_scale<KIND>(p, sp.e, row, gs);
         }
     }
     release_dependents();

@@ -65,6 +65,24 @@ struct Shape {
     static constexpr int kWarps = FUSED ? PQG_WARPS_FUSED : PQG_WARPS_PLAIN;
 };
 
+// Grid cap in waves of resident CTAs for a call of `blocks` blocks, by variant
+// (measured on B200 at the bench workloads): UE8M0 FP8 and the fused kernels
+// run best with up to PQG_WAVES waves; the FP4 kinds with 4; the fp32-scale
+// plain kinds with 2, unless the call is long (>= 24 waves of blocks, e.g.
+// the 65536-row sweeps), where 8 win again.
+#ifndef PQG_WAVES_FP4
+#define PQG_WAVES_FP4 4
+#endif
+#ifndef PQG_WAVES_FP32
+#define PQG_WAVES_FP32 2
+#endif
+template <Kind KIND, bool FUSED>
+inline uint64_t grid_waves(uint64_t blocks, uint64_t wave) {
+    if (FUSED || KIND == Kind::E4M3_UE8M0) return PQG_WAVES;
+    if (is_e2m1(KIND)) return PQG_WAVES_FP4;
+    return blocks >= 24u * wave ? PQG_WAVES : PQG_WAVES_FP32;
+}
+
 template <typename In, int G, Kind KIND, bool FUSED, bool MULTI>
 cudaError_t launch_variant(const LaunchArgs &a) {
     using Sh = Shape<FUSED, MULTI>;
@@ -102,7 +120,8 @@ cudaError_t launch_variant(const LaunchArgs &a) {
     if (a.expected_strips < wave * Sh::kWarps * Sh::kItems) p.items = 1;
     const uint64_t per_cta = static_cast<uint64_t>(Sh::kWarps) * p.items;
     uint64_t ctas = (a.expected_strips + per_cta - 1) / per_cta;
-    const uint64_t cap = ctas <= wave * PQG_SHORT_WAVES ? wave : wave * PQG_WAVES;
+    const uint64_t cap =
+        ctas <= wave * PQG_SHORT_WAVES ? wave : wave * grid_waves<KIND, FUSED>(ctas, wave);
     if (ctas > cap) ctas = cap;
     if (ctas < 1) ctas = 1;
 

@@ -349,7 +349,10 @@ def run_ours(args, w, rank: int, world: int, local_rank: int) -> dict | None:
     with ClockSampler(dev.index) as clocks:
         start.record(stream)
         if graph is not None:
-            graph.replay()
+            # replay on the capture stream: torch replays on the current stream,
+            # and the events are recorded on `stream`
+            with torch.cuda.stream(stream):
+                graph.replay()
         else:
             for i in range(args.steps):
                 launch(args.warmup + i)

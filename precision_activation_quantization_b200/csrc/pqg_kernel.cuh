@@ -2,7 +2,8 @@
 //
 // One kernel body, specialised at compile time on what changes the inner loop:
 // input dtype, group size G, output/scale kind (E4M3 + fp32 scale, E4M3 +
-// UE8M0 scale, INT8 + fp32 scale) and the fused SiLU-and-mul prologue.  What
+// UE8M0 scale, INT8 + fp32 scale, MXFP4 = E2M1 + UE8M0, NVFP4 = E2M1 + E4M3
+// block scale) and the fused SiLU-and-mul prologue.  What
 // changes only once per group (the scale layout) or once per CTA (flat or
 // masked dispatch) is a runtime field of the parameter block.  The variant axes
 // are those of the sglang PR #30924 report, "[JIT] Trait-driven
@@ -20,8 +21,8 @@
 // row of any strip; skewed masked_m cannot leave CTAs idle.
 //
 // Memory-level parallelism.  A warp takes ITEMS strips per chunk and issues
-// all of the chunk's 32-byte loads before any arithmetic; with about 40
-// resident warps per SM (register-light kernel) that keeps the HBM queues full.
+// all of the chunk's 32-byte loads before any arithmetic; with 32-48 resident
+// warps per SM (register-light kernel) that keeps the HBM queues full.
 // Keeping a second chunk in flight was measured slower both ways it was tried:
 // in registers (double-buffering) and in shared memory (cp.async stages), the
 // extra registers and instructions cost more warps than the prefetch won.
@@ -840,8 +841,9 @@ __device__ __forceinline__ void quantize_chunk(const Chunk<ITEMS, FUSED> &ch, co
 // ---------------------------------------------------------------------------
 
 // Resident CTAs per SM the register allocation must allow (0: no constraint).
-// The fp32-scale plain variants run best at 5 (<= 51 registers) and flat NVFP4
-// at 6 (<= 40 registers, no spills); the rest need no constraint.
+// The fp32-scale plain variants run best at 5 (they take 46-48 registers; a
+// bound of 6 spills and was measured no better) and flat NVFP4 at 6 (<= 40
+// registers, no spills); the rest need no constraint.
 #ifndef PQG_MIN_BLOCKS_FP32
 #define PQG_MIN_BLOCKS_FP32 5
 #endif

@@ -1,4 +1,5 @@
-// Instantiates the fp16-input half of the kernel family (18 variants).
+// Instantiates the fp16-input half of the kernel family (52 strip-kernel and
+// 18 per-token variants).
 #include "pqg_launch.cuh"
 
 namespace pqg {

@@ -283,8 +283,7 @@ __device__ __forceinline__ uint32_t e2m1x8(float a0, float a1, float b0, float b
 // fp32 x/s for every x; 1 leaves q within an ulp of it, and exhaustive CPU
 // checks found the E4M3 and INT8 codes of that q equal to the codes of
 // RN(x/s) for every bf16 / fp16 x and every fp32 s (all significand pairs,
-// every binade of x/s that yields a nonzero code).  The strip kernel uses 1,
-// the per-token row kernel 2 (measured faster there).
+// every binade of x/s that yields a nonzero code).  Both kernels use 1.
 #ifndef PQG_DIV_STEPS
 #define PQG_DIV_STEPS 1
 #endif

@@ -22,10 +22,6 @@ namespace pqg {
 
 constexpr int kRowThreads = 256;  // 8 warps per CTA
 
-// Markstein corrections per code of the row kernel (see div_rn2).
-#ifndef PQG_ROW_DIV_STEPS
-#define PQG_ROW_DIV_STEPS 2
-#endif
 
 // The scale of row `row` of expert e.  One group per row: row-major,
 // column-major and packed all put it at element / word `row` of the expert's
@@ -138,12 +134,12 @@ __global__ void __launch_bounds__(kRowThreads)
                 if (slot < nslots) {
                     uint32_t w[4];
                     if constexpr (FUSED) {
-                        encode16<KIND, PQG_ROW_DIV_STEPS>(v[j], gs, w);
+                        encode16<KIND>(v[j], gs, w);
                     } else {
                         float vj[16];
 #pragma unroll
                         for (int i = 0; i < 8; ++i) widen2<In>(x[j][i], vj[2 * i], vj[2 * i + 1]);
-                        encode16<KIND, PQG_ROW_DIV_STEPS>(vj, gs, w);
+                        encode16<KIND>(vj, gs, w);
                     }
                     store16B(dst + slot * 16u, w[0], w[1], w[2], w[3]);
                 }

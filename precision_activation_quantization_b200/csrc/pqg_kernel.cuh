@@ -226,29 +226,10 @@ __device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
     return r;
 }
 
-// Packed pair of OCP E2M1 codes: `lo` in bits 0-3, `hi` in bits 4-7.  Round to
-// nearest even; satfinite clamps to +-6 (never reached: |t| <= 6 here).
-__device__ __forceinline__ uint32_t e2m1x2(float lo, float hi) {
-    uint32_t r;
-    asm("{\n\t.reg .b8 t;\n\tcvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\tcvt.u32.u8 %0, t;\n\t}"
-        : "=r"(r)
-        : "f"(hi), "f"(lo));
-    return r;
-}
-
-// FP4 code bytes packed by a vector move (1) or by shifts (0).
-#ifndef PQG_E2M1_VECPACK
-#define PQG_E2M1_VECPACK 1
-#endif
-// E4M3 code pairs packed by a vector move (1) or by shift/or (0).
-#ifndef PQG_E4M3_VECPACK
-#define PQG_E4M3_VECPACK 1
-#endif
-
 // Four E4M3 codes as one word, (a0, a1) in the low half: two conversions and
-// a vector move.
+// a vector move (measured faster than shift/or: the assembler places the
+// halves).
 __device__ __forceinline__ uint32_t e4m3x4(float a0, float a1, float b0, float b1) {
-#if PQG_E4M3_VECPACK
     uint32_t r;
     asm("{\n\t.reg .b16 p, q;\n\t"
         "cvt.rn.satfinite.e4m3x2.f32 p, %2, %1;\n\t"
@@ -257,14 +238,13 @@ __device__ __forceinline__ uint32_t e4m3x4(float a0, float a1, float b0, float b
         : "=r"(r)
         : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
     return r;
-#else
-    return e4m3x2(a0, a1) | (e4m3x2(b0, b1) << 16);
-#endif
 }
 
-// Eight E2M1 codes (four pairs, pair k from (v[2k], v[2k+1])) as one word:
-// the four code bytes are packed by a vector move, so the assembler is free to
-// place each conversion's byte.
+// Eight OCP E2M1 codes as one word: pair k = (a_k lo, a_k hi) becomes byte k,
+// the first of the pair in bits 0-3 and the second in bits 4-7; round to
+// nearest even, satfinite clamps to +-6 (MXFP4 never reaches it; NVFP4 can).
+// The four bytes are joined by a vector move, so the assembler places each
+// conversion's byte (measured faster than shift/or and than byte permutes).
 __device__ __forceinline__ uint32_t e2m1x8(float a0, float a1, float b0, float b1, float c0,
                                            float c1, float d0, float d1) {
     uint32_t r;
@@ -456,21 +436,11 @@ __device__ __forceinline__ void encode16(const float (&v)[16], const GroupScale 
         const float2 m2 = make_float2(gs.mult, gs.mult);
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
-#if PQG_E2M1_VECPACK
             float2 t[4];
 #pragma unroll
             for (int k = 0; k < 4; ++k)
                 t[k] = __fmul2_rn(make_float2(v[8 * j + 2 * k], v[8 * j + 2 * k + 1]), m2);
             w[j] = e2m1x8(t[0].x, t[0].y, t[1].x, t[1].y, t[2].x, t[2].y, t[3].x, t[3].y);
-#else
-            uint32_t word = 0;
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const float2 t = __fmul2_rn(make_float2(v[8 * j + 2 * k], v[8 * j + 2 * k + 1]), m2);
-                word |= e2m1x2(t.x, t.y) << (8 * k);
-            }
-            w[j] = word;
-#endif
         }
     } else if constexpr (KIND == Kind::E4M3_UE8M0) {
         const float2 m2 = make_float2(gs.mult, gs.mult);
@@ -693,12 +663,6 @@ __device__ __forceinline__ void load_chunk(Chunk<ITEMS, FUSED> &ch, uint32_t s, 
     }
 }
 
-// UE8M0 exponents of the 128x4 tiled layout stored as one word per 4 groups
-// (1; the scale buffer is then 4-byte aligned) or byte by byte (0).
-#ifndef PQG_TILED_WORDS
-#define PQG_TILED_WORDS 1
-#endif
-
 // bf16 UE8M0 through the mixed-precision FMA path (1) or by widening (0).
 #ifndef PQG_UE8M0_MIXED
 #define PQG_UE8M0_MIXED 1
@@ -727,7 +691,6 @@ __device__ __forceinline__ void quantize_strip(const uint32_t (&x)[8], const uin
         gs.e8 = KIND == Kind::E2M1_UE8M0 ? ue8m0_exponent_e2m1(amax) : ue8m0_exponent(amax);
         const uint16_t p2 = static_cast<uint16_t>((254u - gs.e8) << 7);  // bf16 2^(127-e)
         if constexpr (KIND == Kind::E2M1_UE8M0) {
-#if PQG_E2M1_VECPACK
             float t[16];
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
@@ -736,15 +699,6 @@ __device__ __forceinline__ void quantize_strip(const uint32_t (&x)[8], const uin
             }
             w[0] = e2m1x8(t[0], t[1], t[2], t[3], t[4], t[5], t[6], t[7]);
             w[1] = e2m1x8(t[8], t[9], t[10], t[11], t[12], t[13], t[14], t[15]);
-#else
-            w[0] = w[1] = 0u;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const float t0 = mul_bf16_pow2(static_cast<uint16_t>(x[i] & 0xFFFFu), p2);
-                const float t1 = mul_bf16_pow2(static_cast<uint16_t>(x[i] >> 16), p2);
-                w[i >> 2] |= e2m1x2(t0, t1) << (8 * (i & 3));
-            }
-#endif
         } else {
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
@@ -800,19 +754,16 @@ __device__ __forceinline__ void quantize_strip(const uint32_t (&x)[8], const uin
                 reinterpret_cast<uint32_t *>(sc)[static_cast<uint64_t>(g >> 2) * p.mpad + row] =
                     packed_word;
         } else if (p.layout == kTiled128x4) {
-#if PQG_TILED_WORDS
             if constexpr (is_ue8m0(KIND)) {
                 // groups 4j..4j+3 of the row are 4 consecutive bytes of one tile:
-                // one word, its padding bytes already 0
+                // one word, its padding bytes already 0 (the buffer is 4-byte
+                // aligned)
                 if ((g & 3u) == 0u)
                     *reinterpret_cast<uint32_t *>(sc + tile128x4_offset(row, g, p.ng)) =
                         packed_word;
             } else {
-                store_tiled(sc, row, g, p.ng, gs.e8);
+                store_tiled(sc, row, g, p.ng, gs.e8);   // NVFP4 E4M3 block-scale bytes
             }
-#else
-            store_tiled(sc, row, g, p.ng, gs.e8);
-#endif
         } else {
             const uint64_t idx = (p.layout == kRowMajor) ? static_cast<uint64_t>(row) * p.ng + g
                                                          : static_cast<uint64_t>(g) * p.mpad + row;

@@ -291,7 +291,7 @@ def test_per_token_bit_exact(K, kind):
         check_exact(make(M, K, K, kind, in_dtype, seed=K + M))
 
 
-@pytest.mark.parametrize("K", [256, 2048, 7168])
+@pytest.mark.parametrize("K", [80, 256, 2048, 7168, 16384])
 def test_per_token_fused_and_masked(K):
     E, M = 5, 19
     mm = np.array([0, 19, 1, 40, 7], np.int32)

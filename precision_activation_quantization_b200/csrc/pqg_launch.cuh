@@ -8,6 +8,7 @@
 
 #include <atomic>
 #include <cstdint>
+#include <type_traits>
 
 #include "pqg_kernel.cuh"
 #include "pqg_row_kernel.cuh"
@@ -58,10 +59,18 @@ int sm_count(int device);  // cached cudaDevAttrMultiProcessorCount
 // Fused multi-expert (masked) calls take 2 strips per chunk: they are long
 // enough for the deeper chunk to pay (masked 52.9 -> 51.5 us), while a short
 // flat fused call loses warps with work (8.8 -> 9.7 us).
-template <bool FUSED, bool MULTI>
+// Plain bf16 MXFP4 at G = 32 takes 3 strips per chunk (24.86 vs 25.11 us; it
+// stays at 48 registers, where fp16 or G = 64/128 would need 55-62); NVFP4,
+// bounded to 40 registers, loses with 3 (29.2 vs 25.3 us), and masked too.
+#ifndef PQG_ITEMS_MXFP4
+#define PQG_ITEMS_MXFP4 3
+#endif
+template <typename In, Kind KIND, int G, bool FUSED, bool MULTI>
 struct Shape {
-    static constexpr int kItems =
-        FUSED ? (MULTI ? PQG_ITEMS_FUSED_MULTI : PQG_ITEMS_FUSED) : PQG_ITEMS_PLAIN;
+    static constexpr bool kMx32 = KIND == Kind::E2M1_UE8M0 && G == 32 &&
+                                  std::is_same<In, __nv_bfloat16>::value;
+    static constexpr int kItems = FUSED ? (MULTI ? PQG_ITEMS_FUSED_MULTI : PQG_ITEMS_FUSED)
+                                        : (kMx32 ? PQG_ITEMS_MXFP4 : PQG_ITEMS_PLAIN);
     static constexpr int kWarps = FUSED ? PQG_WARPS_FUSED : PQG_WARPS_PLAIN;
 };
 
@@ -85,7 +94,7 @@ inline uint64_t grid_waves(uint64_t blocks, uint64_t wave) {
 
 template <typename In, int G, Kind KIND, bool FUSED, bool MULTI>
 cudaError_t launch_variant(const LaunchArgs &a) {
-    using Sh = Shape<FUSED, MULTI>;
+    using Sh = Shape<In, KIND, G, FUSED, MULTI>;
     constexpr int kThreads = Sh::kWarps * 32;
     auto kernel = quant_kernel<In, G, KIND, FUSED, Sh::kItems, Sh::kWarps, MULTI>;
 

@@ -8,12 +8,13 @@
 // A row is shared by WPR warps (1, 2, 4 or 8, chosen at launch so that a
 // thread holds at most SLOTS 16-element slots).  Lanes read consecutive
 // 32-byte slots, so a warp's loads cover 1 KB contiguous.  The row absmax is a
-// warp xor-reduction, then (WPR > 1) one exchange through shared memory.  The
-// partials are double-buffered by iteration parity, so one __syncthreads per
-// row iteration is enough.  Values stay in registers between the reduction and
-// the quantization, so every input byte is read once.  Rows come from the same
-// expert table as the strip kernel (counting rows instead of strips), so flat,
-// batched and masked dispatch and the fused SiLU-and-mul all work unchanged.
+// warp xor-reduction, then (WPR > 1) one exchange through shared memory behind
+// a named barrier of the row's own warps.  The partials are double-buffered by
+// iteration parity, so one barrier per row iteration is enough.  Values stay in
+// registers between the reduction and the quantization, so every input byte is
+// read once.  Rows come from the same expert table as the strip kernel
+// (counting rows instead of strips), so flat, batched and masked dispatch and
+// the fused SiLU-and-mul all work unchanged.
 #pragma once
 
 #include "pqg_kernel.cuh"
@@ -120,7 +121,10 @@ __global__ void __launch_bounds__(kRowThreads)
         for (int o = 1; o < 32; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
         if (wpr > 1) {
             if (lane == 0) partial[parity][warp] = amax;
-            __syncthreads();
+            // only this row's warps meet: named barrier 1 + sub (0 belongs to
+            // __syncthreads) over wpr warps, so the CTA's rows do not wait on
+            // one another (measured 31.25 -> 30.29 us at K = 7168)
+            asm volatile("bar.sync %0, %1;" ::"r"(1u + sub), "r"(wpr * 32u) : "memory");
             for (uint32_t w = 0; w < wpr; ++w) amax = fmaxf(amax, partial[parity][sub * wpr + w]);
         }
 

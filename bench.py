@@ -55,6 +55,7 @@ def workloads():
         "mxfp4": lambda: inputs.mxfp4(),
         "nvfp4": lambda: inputs.nvfp4(),
         "fused": lambda: inputs.fused(),
+        "fused_7168": lambda: inputs.fused(M=4096, K=7168),
         "masked": lambda: inputs.masked(),
         "masked_decode": lambda: inputs.masked(decode=True),
         "sweep_65536_bf16_e4m3_g128": lambda: inputs.sweep(65536),

@@ -131,6 +131,11 @@ def test_fused_full_size():
     print("fused flips", stats)
 
 
+def test_fused_hidden_size():
+    """Fused SiLU-and-mul at the hidden size: [4096, 2 x 7168]."""
+    check_fused(inputs.fused(M=4096, K=7168))
+
+
 def test_masked_full_size():
     w = inputs.masked()
     stats = check_fused(w)

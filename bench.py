@@ -27,6 +27,7 @@ import datetime
 import hashlib
 import json
 import os
+import re
 import statistics
 import sys
 import threading
@@ -115,17 +116,29 @@ def kernel_of(w) -> str:
     return "row" if w.group == w.K and w.group not in (16, 32, 64, 128) else "strip"
 
 
+_C_TOKENS = re.compile(r'("(?:\\.|[^"\\\n])*"|\'(?:\\.|[^\'\\\n])*\')|//[^\n]*|/\*.*?\*/',
+                       re.DOTALL)
+
+
+def code_only(text: str) -> str:
+    """C/C++ source without its comments, blank lines and trailing blanks
+    (string and character literals kept), so that editing a comment leaves the
+    digest below unchanged."""
+    text = _C_TOKENS.sub(lambda m: m.group(1) or "", text)
+    return "\n".join(l.rstrip() for l in text.splitlines() if l.strip())
+
+
 def source_digest(kernel: str = "strip") -> str:
-    """sha256 over the CUDA sources a kernel is built from (the strip kernel does
-    not include the per-token row kernel's file), to tell whether stored ncu
-    counters still apply."""
+    """sha256 over the code of the CUDA sources a kernel is built from (the
+    strip kernel does not include the per-token row kernel's file), to tell
+    whether stored ncu counters still apply."""
     csrc = os.path.join(ROOT, "precision_activation_quantization_b200", "csrc")
     h = hashlib.sha256()
     for f in sorted(os.listdir(csrc)):
         if kernel == "strip" and f == "pqg_row_kernel.cuh":
             continue
-        with open(os.path.join(csrc, f), "rb") as fh:
-            h.update(f.encode() + fh.read())
+        with open(os.path.join(csrc, f), encoding="utf-8") as fh:
+            h.update(f.encode() + code_only(fh.read()).encode())
     return h.hexdigest()
 
 

@@ -100,11 +100,15 @@ inline uint64_t grid_waves(uint64_t blocks, uint64_t wave) {
     return blocks >= 24u * wave ? PQG_WAVES : PQG_WAVES_FP32;
 }
 
-template <typename In, int G, Kind KIND, bool FUSED, bool MULTI>
+// ITEMS_SEL > 0 overrides the variant's strips per chunk (the long flat fused
+// calls, see launch_kind).
+template <typename In, int G, Kind KIND, bool FUSED, bool MULTI, int ITEMS_SEL = 0>
 cudaError_t launch_variant(const LaunchArgs &a) {
     using Sh = Shape<In, KIND, G, FUSED, MULTI>;
-    constexpr int kThreads = Sh::kWarps * 32;
-    auto kernel = quant_kernel<In, G, KIND, FUSED, Sh::kItems, Sh::kWarps, MULTI>;
+    constexpr int kItems = ITEMS_SEL > 0 ? ITEMS_SEL : Sh::kItems;
+    constexpr int kWarps = Sh::kWarps;
+    constexpr int kThreads = kWarps * 32;
+    auto kernel = quant_kernel<In, G, KIND, FUSED, kItems, kWarps, MULTI>;
 
     // Resident CTAs per SM, queried once per variant without and with the
     // largest shared-memory expert table (more than 32 experts).
@@ -133,9 +137,9 @@ cudaError_t launch_variant(const LaunchArgs &a) {
     // taken round-robin, so any real total is covered.
     const uint64_t wave = static_cast<uint64_t>(sm_count(device)) * blocks_per_sm;
     Params p = a.p;
-    p.items = Sh::kItems;
-    if (a.expected_strips < wave * Sh::kWarps * Sh::kItems) p.items = 1;
-    const uint64_t per_cta = static_cast<uint64_t>(Sh::kWarps) * p.items;
+    p.items = kItems;
+    if (a.expected_strips < wave * kWarps * kItems) p.items = 1;
+    const uint64_t per_cta = static_cast<uint64_t>(kWarps) * p.items;
     uint64_t ctas = (a.expected_strips + per_cta - 1) / per_cta;
     const uint64_t cap =
         ctas <= wave * PQG_SHORT_WAVES ? wave : wave * grid_waves<KIND, FUSED>(ctas, wave);
@@ -158,9 +162,20 @@ cudaError_t launch_variant(const LaunchArgs &a) {
 template <typename In, int G, Kind KIND>
 cudaError_t launch_kind(const LaunchArgs &a) {
     const bool multi = a.p.experts > 1;
-    if (a.fused)
-        return multi ? launch_variant<In, G, KIND, true, true>(a)
-                     : launch_variant<In, G, KIND, true, false>(a);
+    if (a.fused) {
+        if (multi) return launch_variant<In, G, KIND, true, true>(a);
+        // A long flat fused call (4 or more waves of 1-strip work at 48 warps
+        // per SM) runs a variant compiled for 2 strips per chunk: [4096, 2 x
+        // 7168] 26.4 -> 24.6 us.  Short calls keep the 1-strip variant, whose
+        // lower register count holds more CTAs ([4096, 2 x 2048]: 8.8 us
+        // against 10.4 us with the 2-strip build).
+        int device = 0;
+        cudaError_t err = cudaGetDevice(&device);
+        if (err != cudaSuccess) return err;
+        const uint64_t long_call = 4ull * static_cast<uint64_t>(sm_count(device)) * 48u;
+        return a.expected_strips >= long_call ? launch_variant<In, G, KIND, true, false, 2>(a)
+                                              : launch_variant<In, G, KIND, true, false>(a);
+    }
     return multi ? launch_variant<In, G, KIND, false, true>(a)
                  : launch_variant<In, G, KIND, false, false>(a);
 }

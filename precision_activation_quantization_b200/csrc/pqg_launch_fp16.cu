@@ -1,4 +1,4 @@
-// Instantiates the fp16-input half of the kernel family (52 strip-kernel and
+// Instantiates the fp16-input half of the kernel family (65 strip-kernel and
 // 18 per-token variants).
 #include "pqg_launch.cuh"
 

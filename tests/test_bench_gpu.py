@@ -28,8 +28,11 @@ def test_graph_replay_is_timed_on_its_stream(workload):
     calls already hide behind the device, so the graph cannot be much faster
     than stream launches (it can be slower: the replay loses some of the
     programmatic-launch overlap), and neither beats the HBM roofline."""
-    eager = bench("--workload", workload, "--steps", "100")
+    # Two stream-launch runs, compared by the faster: one process on a busy
+    # host can measure a short call a third slower than the next one does.
+    eager = [bench("--workload", workload, "--steps", "100") for _ in range(2)]
     graph = bench("--workload", workload, "--steps", "100", "--graph")
     assert graph["gpu_launches"] == 100
-    assert graph["ms_per_step"] >= 0.8 * eager["ms_per_step"]
-    assert graph["roofline"]["frac"] < 1.2 and eager["roofline"]["frac"] < 1.2
+    best = min(e["ms_per_step"] for e in eager)
+    assert graph["ms_per_step"] >= 0.8 * best
+    assert graph["roofline"]["frac"] < 1.2 and all(e["roofline"]["frac"] < 1.2 for e in eager)

@@ -136,6 +136,31 @@ def test_fused_hidden_size():
     check_fused(inputs.fused(M=4096, K=7168))
 
 
+# A flat fused call of at least 4 waves x 48 strips per SM (28416 strips on
+# 148 SMs) takes two strips per warp chunk; the hidden-size call above is one.
+# These cover the other input type and output kinds of that variant, on a
+# ragged K (14.25 strips per row): [2304, 2 x 7296] is 34560 strips.
+LONG_FUSED = [  # (in_dtype, G, kind)
+    ("fp16", 128, ("e4m3", "ue8m0", "col")),
+    ("bf16", 128, ("e4m3", "fp32", "row")),
+    ("fp16", 64, ("int8", "fp32", "col")),
+    ("bf16", 32, ("e2m1", "ue8m0", "tile128x4")),
+]
+
+
+@pytest.mark.parametrize("in_dtype,G,kind", LONG_FUSED,
+                         ids=lambda v: v if isinstance(v, str) else str(v) if isinstance(v, int)
+                         else "_".join(v))
+def test_fused_long_call_variants(in_dtype, G, kind):
+    check_fused(make(2304, 7296, G, kind, in_dtype, fused=True, seed=G + 71),
+                max_flip_frac=1e-3)
+
+
+def test_fused_long_call_nvfp4():
+    check_fused(make_nv(2304, 7296, 2.625, "tile128x4", "fp16", fused=True, seed=72),
+                max_flip_frac=1e-3)
+
+
 def test_masked_full_size():
     w = inputs.masked()
     stats = check_fused(w)

@@ -35,6 +35,12 @@ MUTANTS = {
                                "int64_t idx = (e * M + m) * ng;"),
     "fused_up_reads_gate": ("float up = pqgo_decode(xrow[K + g * G + i], in_fp16);",
                             "float up = pqgo_decode(xrow[g * G + i], in_fp16);"),
+    "fused_gate_reads_up": ("float x = pqgo_decode(xrow[g * G + i], in_fp16);",
+                            "float x = pqgo_decode(xrow[(fused ? K : 0) + g * G + i], in_fp16);"),
+    "nvfp4_fused_up_reads_gate": ("float up = pqgo_decode(xrow[K + b * G + i], in_fp16);",
+                                  "float up = pqgo_decode(xrow[b * G + i], in_fp16);"),
+    "nvfp4_fused_gate_reads_up": ("float x = pqgo_decode(xrow[b * G + i], in_fp16);",
+                                  "float x = pqgo_decode(xrow[(fused ? K : 0) + b * G + i], in_fp16);"),
     "silu_wrong_sign": ("double silu = g / (1.0 + exp(-g));",
                         "double silu = g / (1.0 + exp(g));"),
     "packed_padding_not_zeroed": ("((uint8_t *)scales)[word * 4 + b] = 0;", ";"),

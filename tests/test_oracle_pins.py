@@ -616,6 +616,32 @@ def test_fused_gate_is_first_half():
     assert not np.array_equal(s, s2)
 
 
+@pytest.mark.parametrize("in_dtype", ["bf16", "fp16"])
+@pytest.mark.parametrize("fmt", [
+    dict(group=128, out_dtype="e4m3", scale_fmt="ue8m0", layout="col"),
+    dict(group=64, out_dtype="int8", scale_fmt="fp32", layout="row"),
+    dict(group=32, out_dtype="e2m1", scale_fmt="ue8m0", layout="tile128x4"),
+    dict(group=16, out_dtype="e2m1", scale_fmt="e4m3", layout="row", global_scale=2.625),
+], ids=["e4m3_ue8m0", "int8_fp32", "mxfp4", "nvfp4"])
+def test_fused_equals_plain_where_silu_is_the_identity(fmt, in_dtype):
+    """For gate >= 32, e^-gate < 2^-46, so silu(gate) = gate / (1 + e^-gate)
+    rounds to gate in fp32 and the fused value is gate * up.  With gates that
+    are powers of two that product is exact in the input type, so the fused
+    call must give the plain call's bytes on the products, in every format."""
+    M, K = 6, 256
+    rng = np.random.default_rng(81)
+    gate = np.exp2(rng.integers(5, 9, (M, K))).astype(np.float32)        # 32 .. 256
+    up_bits = inputs.to_bits(inputs.normal((M, K), 82), in_dtype)
+    up = oracle.decode(up_bits, in_dtype)
+    prod_bits = inputs.to_bits(gate * up, in_dtype)
+    assert np.array_equal(oracle.decode(prod_bits, in_dtype), gate * up)  # exact products
+    fused_x = np.concatenate([inputs.to_bits(gate, in_dtype), up_bits], axis=1)
+    qf, sf = oracle.quant(fused_x.reshape(1, M, 2 * K), M=M, K=K, in_dtype=in_dtype,
+                          fused=True, **fmt)
+    qp, sp = oracle.quant(prod_bits.reshape(1, M, K), M=M, K=K, in_dtype=in_dtype, **fmt)
+    assert np.array_equal(qf, qp) and np.array_equal(sf, sp)
+
+
 # --------------------------------------------------------------------------
 # Layouts and masked dispatch (P-10)
 # --------------------------------------------------------------------------

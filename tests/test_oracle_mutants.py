@@ -31,6 +31,14 @@ MUTANTS = {
     "scale_by_reciprocal": (": amax / PQGO_FMAX_E4M3;", ": amax * (1.0f / PQGO_FMAX_E4M3);"),
     "col_layout_transposed": ("int64_t idx = e * ng * mpad + g * mpad + m;",
                               "int64_t idx = e * ng * mpad + m * ng + g;"),
+    "masked_col_plane_unpadded": ("int64_t idx = e * ng * mpad + g * mpad + m;",
+                                  "int64_t idx = e * ng * M + g * mpad + m;"),
+    "masked_packed_plane_unpadded": ("int64_t word = e * nwords * mpad + (g / 4) * mpad + m;",
+                                     "int64_t word = e * nwords * M + (g / 4) * mpad + m;"),
+    "masked_tile_plane_floor": ("int64_t plane = ((M + 127) / 128) * ((ng + 3) / 4) * 512;\n"
+                                "                    ((uint8_t *)scales)[e * plane",
+                                "int64_t plane = (M / 128) * ((ng + 3) / 4) * 512;\n"
+                                "                    ((uint8_t *)scales)[e * plane"),
     "row_layout_drops_group": ("int64_t idx = (e * M + m) * ng + g;",
                                "int64_t idx = (e * M + m) * ng;"),
     "fused_up_reads_gate": ("float up = pqgo_decode(xrow[K + g * G + i], in_fp16);",
@@ -60,6 +68,10 @@ MUTANTS = {
     "nvfp4_zero_scale_unguarded": ("return d == 0.0f ? 0.0f : g / d;", "return g / d;"),
     "nvfp4_nibbles_swapped": ("qrow[(b * G + i) / 2] = (uint8_t)(lo | (hi << 4));",
                               "qrow[(b * G + i) / 2] = (uint8_t)(hi | (lo << 4));"),
+    "nvfp4_masked_col_plane_unpadded": ("scales[e * ng * mpad + b * mpad + m] = sf;",
+                                        "scales[e * ng * M + b * mpad + m] = sf;"),
+    "nvfp4_tile_plane_floor": ("const int64_t plane = ((M + 127) / 128) * ((ng + 3) / 4) * 512;",
+                               "const int64_t plane = (M / 128) * ((ng + 3) / 4) * 512;"),
     "nvfp4_tile_padding_not_zeroed": ("scales[e * plane + tile128x4_offset(m, b, ng)] = 0;", ";"),
 }
 

@@ -722,6 +722,59 @@ def test_masked_rows_untouched_and_full_mask_equals_flat():
     assert np.array_equal(q2, q.reshape(q2.shape))
 
 
+@pytest.mark.parametrize("fmt,layout,elem", [
+    (dict(group=128, scale_fmt="ue8m0"), "col", 1),
+    (dict(group=128, scale_fmt="fp32"), "col", 4),
+    (dict(group=32, scale_fmt="ue8m0"), "packed", 4),
+    (dict(group=16, out_dtype="e2m1", scale_fmt="e4m3", global_scale=2.625), "col", 1),
+], ids=["ue8m0_col", "fp32_col", "packed", "nvfp4_col"])
+def test_masked_planes_are_padded_like_flat_ones(fmt, layout, elem):
+    """With M = 6 rows per expert the column-major and packed planes are
+    ceil4(6) = 8 rows tall, so expert e's plane starts at e times the
+    one-expert plane size, and holds what a flat call on that expert writes
+    for its live rows; padding rows and masked rows keep the sentinel."""
+    E, M, K = 3, 6, 256
+    x = inputs.bf16_bits(inputs.normal((E, M, K), 23))
+    mm = np.array([6, 3, 0], np.int32)
+    _, s = oracle.quant(x, E=E, M=M, K=K, layout=layout, masked_m=mm, **fmt)
+    s = s.view(np.uint8).reshape(E, -1)
+    ng = K // fmt["group"]
+    plane = (ng if layout == "col" else (ng + 3) // 4) * 8 * (elem if layout == "col" else 4)
+    assert s.shape[1] == plane
+    row = (np.arange(plane) // elem) % 8 if layout == "col" else (np.arange(plane) // 4) % 8
+    for e in range(E):
+        _, sf = oracle.quant(x[e], M=M, K=K, layout=layout, **fmt)
+        sf = sf.view(np.uint8).reshape(-1)
+        live = row < mm[e]
+        assert np.array_equal(s[e, live], sf[live])
+        assert (s[e, ~live] == 0xA5).all()
+        assert (sf[row >= M] == 0xA5).all()            # a flat call skips padding rows too
+
+
+@pytest.mark.parametrize("fmt", [
+    dict(group=32, out_dtype="e2m1", scale_fmt="ue8m0"),
+    dict(group=128, scale_fmt="ue8m0"),
+    dict(group=16, out_dtype="e2m1", scale_fmt="e4m3", global_scale=2.625),
+], ids=["mxfp4", "e4m3_ue8m0", "nvfp4"])
+def test_masked_tiled_planes_hold_whole_tiles(fmt):
+    """128x4-tiled scales of 130 rows take two 128-row tiles per column of
+    tiles, so expert e's plane starts at e * 2 * ceil(ng/4) * 512 bytes: a
+    fully live expert's plane equals a flat call's, an empty one is untouched."""
+    E, M, K = 3, 130, 640
+    x = inputs.bf16_bits(inputs.normal((E, M, K), 24))
+    mm = np.array([M, 0, M], np.int32)
+    _, s = oracle.quant(x, E=E, M=M, K=K, layout="tile128x4", masked_m=mm, **fmt)
+    ng = K // fmt["group"]
+    plane = 2 * ((ng + 3) // 4) * 512
+    s = s.view(np.uint8).reshape(-1)
+    assert s.size == E * plane
+    s = s.reshape(E, plane)
+    for e in (0, 2):
+        _, sf = oracle.quant(x[e], M=M, K=K, layout="tile128x4", **fmt)
+        assert np.array_equal(s[e], sf.view(np.uint8).reshape(-1))
+    assert (s[1] == 0xA5).all()
+
+
 def test_oracle_rejects_unsupported_combinations():
     x = np.zeros((1, 4, 256), np.uint16)
     with pytest.raises(ValueError):

@@ -192,6 +192,8 @@ def quant(x, out=None, scales=None, *, M: int | None = None, K: int | None = Non
 
     ``x`` is bf16/fp16, [E, M, K] / [M, K] ([..., 2K] when ``fuse_silu_mul``).
     ``masked_m`` is an int32 CUDA tensor of E row counts (masked dispatch).
+    ``out``, ``scales`` and ``masked_m`` must be contiguous (``scales`` may be the
+    transposed view of a contiguous buffer): the kernel addresses each densely.
     NVFP4 is ``out_dtype="e2m1", scale_fmt="e4m3", group=16`` with
     ``global_scale`` a one-element fp32 CUDA tensor (pqg_quant_nvfp4).
     The kernel runs on ``stream`` (default: torch's current stream).
@@ -225,11 +227,18 @@ def quant(x, out=None, scales=None, *, M: int | None = None, K: int | None = Non
         raise ValueError(f"scales must be {nbytes} bytes for this layout")
     if not (out.is_cuda and scales.is_cuda and out.device == x.device == scales.device):
         raise ValueError("x, out and scales must be on the same CUDA device")
+    # the kernel addresses every buffer from its first byte, densely
+    if not out.is_contiguous():
+        raise ValueError("out must be contiguous")
+    if not (scales.is_contiguous()
+            or (scales.dim() >= 2 and scales.transpose(-1, -2).is_contiguous())):
+        raise ValueError("scales must be contiguous, or the transposed view of a contiguous buffer")
     mm_ptr = None
     if masked_m is not None:
         if (masked_m.dtype != torch.int32 or masked_m.device != x.device
-                or masked_m.numel() != E):
-            raise ValueError("masked_m must be an int32 CUDA tensor with one entry per expert")
+                or masked_m.numel() != E or not masked_m.is_contiguous()):
+            raise ValueError("masked_m must be a contiguous int32 CUDA tensor with one entry "
+                             "per expert")
         mm_ptr = masked_m.data_ptr()
     if stream is None:
         stream = torch.cuda.current_stream(x.device)

@@ -272,6 +272,32 @@ def test_torch_helper_matches_raw_call():
         pqg.quant(x, group=128, out_dtype="int8", scale_fmt="ue8m0")
 
 
+def test_torch_helper_rejects_strided_buffers():
+    """The kernel writes and reads each buffer densely from its first byte, so
+    a strided view of the right size is refused before the launch; the
+    transposed view of a column-major scale buffer is accepted."""
+    M, K = 64, 1024
+    x = torch.randn(M, K, device="cuda").to(torch.bfloat16)
+    out, sc = pqg.allocate_outputs(M, K, 128, scale_fmt="fp32", layout="col", device="cuda")
+    before = pqg.pqg_launch_count()
+    wide = torch.empty(1, M, 2 * K, dtype=torch.float8_e4m3fn, device="cuda")
+    with pytest.raises(ValueError, match="out must be contiguous"):
+        pqg.quant(x, wide[..., ::2], sc, group=128, scale_fmt="fp32", layout="col")
+    tall = torch.empty(1, 2 * (K // 128), M, dtype=torch.float32, device="cuda")
+    with pytest.raises(ValueError, match="scales must be contiguous"):
+        pqg.quant(x, out, tall[:, ::2], group=128, scale_fmt="fp32", layout="col")
+    xe = torch.randn(4, M, K, device="cuda").to(torch.bfloat16)
+    counts = torch.full((8,), M, dtype=torch.int32, device="cuda")
+    with pytest.raises(ValueError, match="masked_m must be a contiguous"):
+        pqg.quant(xe, group=128, masked_m=counts[::2])
+    assert pqg.pqg_launch_count() == before
+    q, s = pqg.quant(x, out, sc.transpose(-1, -2), group=128, scale_fmt="fp32", layout="col")
+    q2, s2 = pqg.quant(x, group=128, scale_fmt="fp32", layout="col")
+    torch.cuda.synchronize()
+    assert torch.equal(q.view(torch.uint8), q2.view(torch.uint8))
+    assert torch.equal(sc, s2)
+
+
 # --------------------------------------------------------------------------
 # the balanced scheduler and its expert table
 # --------------------------------------------------------------------------

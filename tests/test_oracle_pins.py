@@ -16,6 +16,7 @@ import os
 import numpy as np
 import pytest
 import torch
+from hypothesis import given, settings, strategies as st
 
 import oracle
 from precision_activation_quantization_b200 import inputs
@@ -811,3 +812,67 @@ def test_inputs_are_deterministic_and_shaped():
     assert m.x.shape == (4, 64, 256) and m.masked_m.min() >= 0 and m.masked_m.max() <= 64
     d = inputs.masked(E=8, M_max=16, K=128, decode=True)
     assert set(np.unique(d.masked_m)) <= {0, 1} and d.expected_m == 1
+
+
+# --------------------------------------------------------------------------
+# Layout properties at random sizes
+# --------------------------------------------------------------------------
+
+
+@st.composite
+def _layout_case(draw):
+    E = draw(st.integers(1, 3))
+    M = draw(st.sampled_from([0, 1, 2, 3, 4, 5, 7, 9, 130]))
+    G = draw(st.sampled_from([32, 64, 128]))
+    ng = draw(st.integers(1, 6))
+    masked = draw(st.booleans())
+    mm = (np.array(draw(st.lists(st.integers(-2, M + 2), min_size=E, max_size=E)), np.int32)
+          if masked else None)
+    return E, M, G, ng, mm, draw(st.sampled_from(["bf16", "fp16"])), draw(st.integers(0, 999))
+
+
+@settings(max_examples=60, deadline=None)
+@given(_layout_case())
+def test_layouts_hold_one_table_at_random_sizes(case):
+    """Every layout holds the row-major table at its defined position: column-
+    major S[g][m] over ceil4(M) rows, packed words W[j][m] with group 4j+b in
+    byte b, and 128x4 tiles; packed and tiled padding groups of live rows are
+    0, and nothing else outside the live rows is written.  Codes do not depend
+    on the layout, and masked-off rows keep the sentinel."""
+    E, M, G, ng, mm, in_dtype, seed = case
+    K = ng * G
+    x = inputs.to_bits(inputs.normal((E, M, K), seed) * 4, in_dtype)
+    live = np.full(E, M) if mm is None else np.clip(mm, 0, M)
+    kw = dict(E=E, M=M, K=K, group=G, in_dtype=in_dtype, masked_m=mm)
+    q_row, s_row = oracle.quant(x, scale_fmt="ue8m0", layout="row", **kw)
+    q_row = q_row.reshape(E, M, K)
+    row = s_row.reshape(E, M, ng)
+    mpad, nw, ct = (M + 3) // 4 * 4, (ng + 3) // 4, (ng + 3) // 4
+    for layout in ("col", "packed", "tile128x4"):
+        q, s = oracle.quant(x, scale_fmt="ue8m0", layout=layout, **kw)
+        assert np.array_equal(q.reshape(E, M, K), q_row)
+        s = s.view(np.uint8).reshape(E, -1)
+        want = np.full_like(s, 0xA5)
+        for e in range(E):
+            for m in range(live[e]):
+                for g in range(4 * nw if layout != "col" else ng):
+                    v = row[e, m, g] if g < ng else 0
+                    if layout == "col":
+                        want[e, g * mpad + m] = v
+                    elif layout == "packed":
+                        want[e, ((g // 4) * mpad + m) * 4 + g % 4] = v
+                    else:
+                        r = m % 128
+                        want[e, ((m // 128) * ct + g // 4) * 512 + (r % 32) * 16 + (r // 32) * 4
+                             + g % 4] = v
+        assert np.array_equal(s, want), layout
+    for e in range(E):
+        assert (q_row[e, live[e]:] == 0xA5).all()
+        assert (row[e, live[e]:] == 0xA5).all()
+    _, f_row = oracle.quant(x, scale_fmt="fp32", layout="row", **kw)
+    _, f_col = oracle.quant(x, scale_fmt="fp32", layout="col", **kw)
+    f_row, f_col = f_row.reshape(E, M, ng), f_col.reshape(E, ng, mpad)
+    for e in range(E):
+        n = live[e]
+        assert np.array_equal(f_col[e, :, :n].view(np.uint32), f_row[e, :n].T.view(np.uint32))
+        assert (f_col[e, :, n:].view(np.uint32) == 0xA5A5A5A5).all()

@@ -831,6 +831,28 @@ def _layout_case(draw):
     return E, M, G, ng, mm, draw(st.sampled_from(["bf16", "fp16"])), draw(st.integers(0, 999))
 
 
+def _planes_from_rows(row, live, layout, plane_bytes):
+    """The bytes each expert's scale plane must hold: the row-major byte table
+    `row` [E, M, ng] placed at the layout's defined positions for the live
+    rows (padding groups of those rows 0), the sentinel everywhere else."""
+    E, M, ng = row.shape
+    mpad, nw = (M + 3) // 4 * 4, (ng + 3) // 4
+    want = np.full((E, plane_bytes), 0xA5, np.uint8)
+    for e in range(E):
+        for m in range(live[e]):
+            for g in range(4 * nw if layout != "col" else ng):
+                v = row[e, m, g] if g < ng else 0
+                if layout == "col":
+                    want[e, g * mpad + m] = v
+                elif layout == "packed":
+                    want[e, ((g // 4) * mpad + m) * 4 + g % 4] = v
+                else:
+                    r = m % 128
+                    want[e, ((m // 128) * nw + g // 4) * 512 + (r % 32) * 16 + (r // 32) * 4
+                         + g % 4] = v
+    return want
+
+
 @settings(max_examples=60, deadline=None)
 @given(_layout_case())
 def test_layouts_hold_one_table_at_random_sizes(case):
@@ -847,28 +869,15 @@ def test_layouts_hold_one_table_at_random_sizes(case):
     q_row, s_row = oracle.quant(x, scale_fmt="ue8m0", layout="row", **kw)
     q_row = q_row.reshape(E, M, K)
     row = s_row.reshape(E, M, ng)
-    mpad, nw, ct = (M + 3) // 4 * 4, (ng + 3) // 4, (ng + 3) // 4
     for layout in ("col", "packed", "tile128x4"):
         q, s = oracle.quant(x, scale_fmt="ue8m0", layout=layout, **kw)
         assert np.array_equal(q.reshape(E, M, K), q_row)
         s = s.view(np.uint8).reshape(E, -1)
-        want = np.full_like(s, 0xA5)
-        for e in range(E):
-            for m in range(live[e]):
-                for g in range(4 * nw if layout != "col" else ng):
-                    v = row[e, m, g] if g < ng else 0
-                    if layout == "col":
-                        want[e, g * mpad + m] = v
-                    elif layout == "packed":
-                        want[e, ((g // 4) * mpad + m) * 4 + g % 4] = v
-                    else:
-                        r = m % 128
-                        want[e, ((m // 128) * ct + g // 4) * 512 + (r % 32) * 16 + (r // 32) * 4
-                             + g % 4] = v
-        assert np.array_equal(s, want), layout
+        assert np.array_equal(s, _planes_from_rows(row, live, layout, s.shape[1])), layout
     for e in range(E):
         assert (q_row[e, live[e]:] == 0xA5).all()
         assert (row[e, live[e]:] == 0xA5).all()
+    mpad = (M + 3) // 4 * 4
     _, f_row = oracle.quant(x, scale_fmt="fp32", layout="row", **kw)
     _, f_col = oracle.quant(x, scale_fmt="fp32", layout="col", **kw)
     f_row, f_col = f_row.reshape(E, M, ng), f_col.reshape(E, ng, mpad)
@@ -876,3 +885,27 @@ def test_layouts_hold_one_table_at_random_sizes(case):
         n = live[e]
         assert np.array_equal(f_col[e, :, :n].view(np.uint32), f_row[e, :n].T.view(np.uint32))
         assert (f_col[e, :, n:].view(np.uint32) == 0xA5A5A5A5).all()
+
+
+@settings(max_examples=40, deadline=None)
+@given(_layout_case(), st.sampled_from([1.0, 2.625, 896.0]), st.booleans())
+def test_nvfp4_layouts_hold_one_table_at_random_sizes(case, g, fused):
+    """The same property for NVFP4's E4M3 block-scale bytes (blocks of 16,
+    row, column-major and tiled), which its own loop writes, fused or not."""
+    E, M, _, ng, mm, in_dtype, seed = case
+    K = ng * 16
+    x = inputs.to_bits(inputs.normal((E, M, 2 * K if fused else K), seed) * 4, in_dtype)
+    live = np.full(E, M) if mm is None else np.clip(mm, 0, M)
+    kw = dict(E=E, M=M, K=K, group=16, in_dtype=in_dtype, out_dtype="e2m1", scale_fmt="e4m3",
+              fused=fused, masked_m=mm, global_scale=g)
+    q_row, s_row = oracle.quant(x, layout="row", **kw)
+    q_row = q_row.reshape(E, M, K // 2)
+    row = s_row.reshape(E, M, ng)
+    for layout in ("col", "tile128x4"):
+        q, s = oracle.quant(x, layout=layout, **kw)
+        assert np.array_equal(q.reshape(E, M, K // 2), q_row)
+        s = s.view(np.uint8).reshape(E, -1)
+        assert np.array_equal(s, _planes_from_rows(row, live, layout, s.shape[1])), layout
+    for e in range(E):
+        assert (q_row[e, live[e]:] == 0xA5).all()
+        assert (row[e, live[e]:] == 0xA5).all()

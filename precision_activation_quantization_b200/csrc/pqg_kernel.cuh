@@ -17,8 +17,9 @@
 // log2(L)-step xor-shuffle.  The strips of all experts (rows < masked_m[e]
 // only) form one sequence, cut into blocks of WARPS x ITEMS strips that the
 // CTAs take round-robin.  With several experts each CTA first prefix-sums the
-// per-expert strip counts in shared memory, so a warp can find the expert and
-// row of any strip; skewed masked_m cannot leave CTAs idle.
+// per-expert strip counts (in each warp's registers up to 32 experts, in
+// shared memory beyond), so a warp can find the expert and row of any strip;
+// skewed masked_m cannot leave CTAs idle.
 //
 // Memory-level parallelism.  A warp takes ITEMS strips per chunk and issues
 // all of the chunk's 32-byte loads before any arithmetic; with 32-48 resident

@@ -909,3 +909,31 @@ def test_nvfp4_layouts_hold_one_table_at_random_sizes(case, g, fused):
     for e in range(E):
         assert (q_row[e, live[e]:] == 0xA5).all()
         assert (row[e, live[e]:] == 0xA5).all()
+
+
+@settings(max_examples=40, deadline=None)
+@given(_layout_case(), st.sampled_from([
+    dict(out_dtype="e4m3", scale_fmt="ue8m0", layout="packed"),
+    dict(out_dtype="e4m3", scale_fmt="fp32", layout="col"),
+    dict(out_dtype="int8", scale_fmt="fp32", layout="row"),
+    dict(out_dtype="e2m1", scale_fmt="ue8m0", layout="tile128x4"),
+    dict(out_dtype="e2m1", scale_fmt="e4m3", layout="col", global_scale=2.625),
+]))
+def test_fused_equals_plain_where_silu_is_the_identity_at_random_sizes(case, fmt):
+    """The identity of test_fused_equals_plain_where_silu_is_the_identity
+    (power-of-two gates >= 32, so silu(gate) * up = gate * up exactly) under
+    random experts, rows, masks, layouts and formats."""
+    E, M, G, ng, mm, in_dtype, seed = case
+    G = 16 if fmt["scale_fmt"] == "e4m3" else G
+    K = ng * G
+    rng = np.random.default_rng(seed)
+    gate = np.exp2(rng.integers(5, 9, (E, M, K))).astype(np.float32)
+    up_bits = inputs.to_bits(inputs.normal((E, M, K), seed + 1), in_dtype)
+    prod = gate * oracle.decode(up_bits, in_dtype).reshape(E, M, K)
+    prod_bits = inputs.to_bits(prod, in_dtype)
+    assert np.array_equal(oracle.decode(prod_bits, in_dtype).reshape(E, M, K), prod)
+    fused_x = np.concatenate([inputs.to_bits(gate, in_dtype), up_bits], axis=-1)
+    kw = dict(E=E, M=M, K=K, group=G, in_dtype=in_dtype, masked_m=mm, **fmt)
+    qf, sf = oracle.quant(fused_x, fused=True, **kw)
+    qp, sp = oracle.quant(prod_bits, **kw)
+    assert np.array_equal(qf, qp) and np.array_equal(sf.view(np.uint8), sp.view(np.uint8))

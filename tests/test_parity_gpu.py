@@ -188,10 +188,27 @@ def test_sweep_largest(in_dtype, out_dtype, G):
 # dispatch properties
 # --------------------------------------------------------------------------
 
-def test_expected_m_does_not_change_results():
+EXPECTED_M_CASES = {   # name -> workload factory (E, M, K, masked_m)
+    "e4m3_ue8m0_fused": lambda E, M, K, mm: make(M, K, 128, ("e4m3", "ue8m0", "col"), fused=True,
+                                                 E=E, seed=9, masked_m=mm),
+    "int8_fp32": lambda E, M, K, mm: make(M, K, 64, ("int8", "fp32", "row"), E=E, seed=13,
+                                          masked_m=mm),
+    "per_token": lambda E, M, K, mm: make(M, K, K, ("e4m3", "fp32", "col"), E=E, seed=14,
+                                          masked_m=mm),
+    "mxfp4_fused_tiled": lambda E, M, K, mm: make(M, K, 32, ("e2m1", "ue8m0", "tile128x4"),
+                                                  fused=True, E=E, seed=15, masked_m=mm),
+    "nvfp4_tiled": lambda E, M, K, mm: make_nv(M, K, 2.625, "tile128x4", E=E, seed=16,
+                                               masked_m=mm),
+}
+
+
+@pytest.mark.parametrize("case", list(EXPECTED_M_CASES))
+def test_expected_m_does_not_change_results(case):
+    """expected_m sizes the grid and the strips per warp; the bytes written
+    must not depend on it."""
     E, M, K = 6, 64, 1024
     mm = np.array([64, 3, 0, 17, 64, 40], np.int32)
-    w = make(M, K, 128, ("e4m3", "ue8m0", "col"), fused=True, E=E, seed=9, masked_m=mm)
+    w = EXPECTED_M_CASES[case](E, M, K, mm)
     ref = run_gpu(w, expected_m=1)
     for em in (0, 8, 30, 64, 1000):
         got = run_gpu(w, expected_m=em)

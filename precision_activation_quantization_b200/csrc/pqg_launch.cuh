@@ -63,7 +63,8 @@ int sm_count(int device);  // cached cudaDevAttrMultiProcessorCount
 
 // Fused multi-expert (masked) calls take 2 strips per chunk: they are long
 // enough for the deeper chunk to pay (masked 52.9 -> 51.5 us), while a short
-// flat fused call loses warps with work (8.8 -> 9.7 us).
+// flat fused call loses warps with work (8.8 -> 9.7 us); long flat fused
+// calls take 2 as well (launch_kind picks the variant by call length).
 // Plain bf16 MXFP4 at G = 32 takes 3 strips per chunk (24.86 vs 25.11 us; it
 // stays at 48 registers, where fp16 or G = 64/128 would need 55-62); NVFP4,
 // bounded to 40 registers, loses with 3 (29.2 vs 25.3 us), and masked too.

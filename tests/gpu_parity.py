@@ -64,6 +64,7 @@ def run_oracle(w):
 
 
 def assert_same(gpu, ref, what):
+    gpu, ref = np.ravel(gpu), np.ravel(ref)
     if np.array_equal(gpu, ref):
         return
     bad = np.flatnonzero(gpu != ref)

@@ -248,7 +248,8 @@ def check_fused(w, *, max_flip_frac=1e-4, rel_tol=7e-2, **kw):
         # dequantizes to zero.
         zero = np.broadcast_to(g_sc[..., None] == 0, t.shape)
         if zero.any():
-            assert w.scale_fmt == "e4m3" and (vals[zero] == 0).all()
+            assert w.scale_fmt == "e4m3" and (vals[zero] == 0).all(), \
+                f"{w.name}: nonzero codes in zero blocks"
             bound0 = 6.0 * 2.0 ** -10 / np.float64(np.float32(w.global_scale))
             assert (err[zero] <= bound0 * (1 + 2.0 ** -10)).all(), f"{w.name}: zero blocks"
         # An NVFP4 block scale saturated at 448 leaves t above 6: those codes

@@ -167,3 +167,30 @@ def test_fused_check_catches_a_two_step_e2m1_code(monkeypatch):
     _device_returns(monkeypatch, two_steps)
     with pytest.raises(AssertionError, match="more than one step"):
         check_fused(w, max_flip_frac=1e-3)
+
+
+def test_fused_check_catches_nonzero_packed_padding(monkeypatch):
+    """ng = 5 groups leave bytes 1..3 of each row's second packed word as
+    padding, which must hold 0."""
+    w = _fp8_fused("packed")
+    nw, mpad = 2, (M + 3) // 4 * 4
+
+    def pad(w, q, s):
+        s[((0 * nw + 1) * mpad + 4) * 4 + 2] = 7    # expert 0, word 1, row 4, byte 2
+    _device_returns(monkeypatch, pad)
+    with pytest.raises(AssertionError, match="packed padding bytes must be 0"):
+        check_fused(w)
+
+
+def test_fused_check_catches_codes_in_an_nvfp4_zero_block(monkeypatch):
+    """A block whose scale code is 0 must dequantize to 0: a nonzero code
+    there fails, even though the flip budget would allow one flip."""
+    w = make_nv(M, K, 2.625, "row", fused=True, E=E, seed=6, masked_m=MASK)
+
+    def code(w, q, s):
+        b = int(np.flatnonzero(s.reshape(E, M, K // 16)[0, :5] == 0)[0])   # a zero block
+        m, blk = divmod(b, K // 16)
+        q[(m * K + blk * 16) // 2] = 0x01               # code 0.5: one step from 0
+    _device_returns(monkeypatch, code)
+    with pytest.raises(AssertionError, match="nonzero codes in zero blocks"):
+        check_fused(w, max_flip_frac=1e-3)

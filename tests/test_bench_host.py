@@ -1,5 +1,6 @@
 """Host logic of bench.py that needs no GPU: the source digest that tells
-whether the stored ncu traffic counters still describe the built kernels."""
+whether the stored ncu traffic counters still describe the built kernels, and
+the bench commands the ncu summaries under profiles/ were captured on."""
 import os
 import re
 import sys

@@ -192,8 +192,11 @@ def quant(x, out=None, scales=None, *, M: int | None = None, K: int | None = Non
 
     ``x`` is bf16/fp16, [E, M, K] / [M, K] ([..., 2K] when ``fuse_silu_mul``).
     ``masked_m`` is an int32 CUDA tensor of E row counts (masked dispatch).
-    ``out``, ``scales`` and ``masked_m`` must be contiguous (``scales`` may be the
-    transposed view of a contiguous buffer): the kernel addresses each densely.
+    ``out``, ``scales`` and ``masked_m`` must be contiguous: the kernel addresses
+    each densely.  With the column-wise layouts ("col", "packed") ``scales`` may
+    also be the [.., M_pad, columns] transposed view of its contiguous plane; any
+    other non-contiguous view raises.  The call runs with ``x``'s device current,
+    whichever device is current in the caller.
     NVFP4 is ``out_dtype="e2m1", scale_fmt="e4m3", group=16`` with
     ``global_scale`` a one-element fp32 CUDA tensor (pqg_quant_nvfp4).
     The kernel runs on ``stream`` (default: torch's current stream).
@@ -230,9 +233,16 @@ def quant(x, out=None, scales=None, *, M: int | None = None, K: int | None = Non
     # the kernel addresses every buffer from its first byte, densely
     if not out.is_contiguous():
         raise ValueError("out must be contiguous")
-    if not (scales.is_contiguous()
-            or (scales.dim() >= 2 and scales.transpose(-1, -2).is_contiguous())):
-        raise ValueError("scales must be contiguous, or the transposed view of a contiguous buffer")
+    if not scales.is_contiguous():
+        # only a column-wise layout can be handed over as its [.., M_pad, columns]
+        # transposed view; its underlying buffer must be the dense plane
+        ng = K // group
+        cols = {"col": ng, "packed": (ng + 3) // 4}.get(layout)
+        if (cols is None or scales.dim() < 2 or not scales.transpose(-1, -2).is_contiguous()
+                or scales.shape[-1] != cols or scales.shape[-2] != (M + 3) // 4 * 4):
+            raise ValueError(f"a non-contiguous scales view must be the transposed "
+                             f"[M_pad, groups] view of a contiguous '{layout}' plane; "
+                             f"layout '{layout}' does not match this view")
     mm_ptr = None
     if masked_m is not None:
         if (masked_m.dtype != torch.int32 or masked_m.device != x.device
@@ -242,6 +252,15 @@ def quant(x, out=None, scales=None, *, M: int | None = None, K: int | None = Non
         mm_ptr = masked_m.data_ptr()
     if stream is None:
         stream = torch.cuda.current_stream(x.device)
+    # the library sizes its grid from, and launches on, the current device
+    with torch.cuda.device(x.device):
+        return _launch(x, out, scales, M, E, K, group, in_dtype, out_dtype, scale_fmt, layout,
+                       fuse_silu_mul, mm_ptr, expected_m, global_scale, stream)
+
+
+def _launch(x, out, scales, M, E, K, group, in_dtype, out_dtype, scale_fmt, layout,
+            fuse_silu_mul, mm_ptr, expected_m, global_scale, stream):
+    import torch
     if scale_fmt == "e4m3":
         if (global_scale is None or global_scale.dtype != torch.float32
                 or global_scale.numel() != 1 or global_scale.device != x.device):

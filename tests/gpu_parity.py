@@ -7,6 +7,9 @@ touch, or writes past the buffer, show up as changed sentinel bytes.
 """
 from __future__ import annotations
 
+import json
+import os
+
 import numpy as np
 import torch
 
@@ -135,7 +138,25 @@ def _scale_planes(w, sbytes):
     return f.astype(np.float64), None
 
 
-def check_fused(w, *, max_flip_frac=1e-4, rel_tol=7e-2, **kw):
+CONTRACT_FLIP_FRAC = 1e-4     # fused codes: one-step flips on at most 1e-4 of elements
+SMALL_SAMPLE = 100_000         # below this many elements a looser budget may be passed
+
+
+def _log_flips(w, flips, n_el, scale_flips, budget):
+    """Print the observed flip count, and append it as a JSON line to the file
+    named by PQG_FLIP_LOG when that variable is set."""
+    rec = dict(workload=w.name, E=int(w.E), M=int(w.M), K=int(w.K), group=int(w.group),
+               in_dtype=w.in_dtype, out_dtype=w.out_dtype, scale_fmt=w.scale_fmt,
+               layout=w.layout, elements=int(n_el), flips=flips, flip_frac=flips / max(n_el, 1),
+               scale_flips=scale_flips, budget=budget)
+    print("fused flips", rec)
+    path = os.environ.get("PQG_FLIP_LOG")
+    if path:
+        with open(path, "a") as f:
+            f.write(json.dumps(rec) + "\n")
+
+
+def check_fused(w, *, max_flip_frac=CONTRACT_FLIP_FRAC, rel_tol=7e-2, **kw):
     """Fused contract: UE8M0 bytes equal unless the oracle's amax/448 is within
     2^-20 of a power of two; fp32 scales within 2^-19 relative; codes equal
     except for at most ``max_flip_frac`` of elements (outside groups whose UE8M0
@@ -229,7 +250,13 @@ def check_fused(w, *, max_flip_frac=1e-4, rel_tol=7e-2, **kw):
         step = np.abs(E4M3_RANK[gcodes].astype(np.int64) - E4M3_RANK[rcodes].astype(np.int64))
     assert (step[diff] <= 1).all(), f"{w.name}: a code moved by more than one step"
     frac = diff.sum() / max(n_el, 1)
-    assert frac <= max_flip_frac, f"{w.name}: {frac:.2e} of codes differ (> {max_flip_frac})"
+    # The contract allows one-step flips on at most 1e-4 of elements.  A looser
+    # budget may be passed for small samples only: under 1e5 elements a single
+    # flip at a rounding tie is already 1e-5 or more.  From 1e5 elements up the
+    # contract's 1e-4 applies, whatever budget was passed.
+    budget = max_flip_frac if n_el < SMALL_SAMPLE else min(max_flip_frac, CONTRACT_FLIP_FRAC)
+    _log_flips(w, int(diff.sum()), n_el, int(scale_diff.sum()), budget)
+    assert frac <= budget, f"{w.name}: {frac:.2e} of codes differ (> {budget})"
 
     # dequantized GPU value vs the oracle's y, per element
     vals = (gcodes.view(np.int8).astype(np.float64) if w.out_dtype == "int8"

@@ -1,8 +1,9 @@
 """Host logic of bench.py that needs no GPU: the source digest that tells
-whether the stored ncu traffic counters still describe the built kernels, and
-the bench commands the ncu summaries under profiles/ were captured on."""
+whether the stored ncu traffic counters still describe the built kernels, the
+sample statistics of the timed region, and the bench commands the ncu
+summaries under profiles/ were captured on (listed in profiles/captures.json)."""
+import json
 import os
-import re
 import sys
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -39,23 +40,24 @@ def test_digests_separate_the_two_kernels():
     assert len(strip) == len(row) == 64 and strip != row
 
 
-def test_profile_commands_run_committed_code_on_known_workloads():
-    """Every ncu summary names the bench command it was captured on; that
-    command must be bench.py with flags it accepts and a workload it knows."""
+def test_capture_commands_run_committed_code_on_known_workloads():
+    """Every summary under profiles/ has an entry in captures.json naming the
+    bench command it was captured on; that command must be bench.py with flags
+    it accepts and a workload it knows, and every listed summary must exist."""
     prof = os.path.join(ROOT, "profiles")
+    with open(os.path.join(prof, "captures.json"), encoding="utf-8") as f:
+        caps = json.load(f)["captures"]
     known = set(bench.workloads())
-    seen = 0
-    for name in sorted(os.listdir(prof)):
-        if not name.endswith(".md") or name == "README.md":
-            continue
-        text = open(os.path.join(prof, name), encoding="utf-8").read()
-        cmds = re.findall(r"python bench\.py([^\n#\\]*)", text)
-        assert cmds, f"{name} gives no bench command"
-        for args in cmds:
-            flags = args.split()
-            if "--workload" in flags:
-                assert flags[flags.index("--workload") + 1] in known, (name, args)
-            assert set(f for f in flags if f.startswith("--")) <= {
-                "--kernel-only", "--steps", "--warmup", "--no-cpu-baseline", "--workload"}, (name, args)
-            seen += 1
-    assert seen >= 9
+    listed = {c["summary"] for c in caps}
+    on_disk = {n for n in os.listdir(prof) if n.endswith(".md") and n != "README.md"}
+    assert listed == on_disk, (listed ^ on_disk)
+    for c in caps:
+        flags = c["bench_command"].split()
+        assert flags[:2] == ["python", "bench.py"], c
+        if "--workload" in flags:
+            assert flags[flags.index("--workload") + 1] in known, c
+        assert set(f for f in flags if f.startswith("--")) <= {
+            "--kernel-only", "--steps", "--warmup", "--no-cpu-baseline", "--workload",
+            "--samples"}, c
+        assert "--clock-control none" in c["ncu"], c
+    assert len(caps) >= 9

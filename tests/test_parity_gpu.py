@@ -71,8 +71,10 @@ def test_flat_variants_bit_exact(kind, G, in_dtype):
 @pytest.mark.parametrize("in_dtype", ["bf16", "fp16"])
 def test_fused_variants_within_contract(kind, G, in_dtype):
     for M, K in [(37, 640), (130, 2048)]:
+        # 1e-3 binds only the 23 680-element case; the 266 240-element one is
+        # held to the contract's 1e-4 by check_fused
         check_fused(make(M, K, G, kind, in_dtype, fused=True, seed=M + K + G + 1),
-                    max_flip_frac=1e-3)   # small samples: a handful of flips
+                    max_flip_frac=1e-3)
 
 
 @pytest.mark.parametrize("kind", KINDS, ids=lambda k: "_".join(k))
@@ -127,8 +129,7 @@ def test_flat_hidden_full_size(layout, fmt):
 
 
 def test_fused_full_size():
-    stats = check_fused(inputs.fused())
-    print("fused flips", stats)
+    check_fused(inputs.fused())
 
 
 def test_fused_hidden_size():
@@ -152,19 +153,15 @@ LONG_FUSED = [  # (in_dtype, G, kind)
                          ids=lambda v: v if isinstance(v, str) else str(v) if isinstance(v, int)
                          else "_".join(v))
 def test_fused_long_call_variants(in_dtype, G, kind):
-    check_fused(make(2304, 7296, G, kind, in_dtype, fused=True, seed=G + 71),
-                max_flip_frac=1e-3)
+    check_fused(make(2304, 7296, G, kind, in_dtype, fused=True, seed=G + 71))
 
 
 def test_fused_long_call_nvfp4():
-    check_fused(make_nv(2304, 7296, 2.625, "tile128x4", "fp16", fused=True, seed=72),
-                max_flip_frac=1e-3)
+    check_fused(make_nv(2304, 7296, 2.625, "tile128x4", "fp16", fused=True, seed=72))
 
 
 def test_masked_full_size():
-    w = inputs.masked()
-    stats = check_fused(w)
-    print("masked flips", stats)
+    check_fused(inputs.masked())
 
 
 def test_masked_decode():
@@ -301,8 +298,11 @@ def test_torch_helper_rejects_strided_buffers():
     with pytest.raises(ValueError, match="out must be contiguous"):
         pqg.quant(x, wide[..., ::2], sc, group=128, scale_fmt="fp32", layout="col")
     tall = torch.empty(1, 2 * (K // 128), M, dtype=torch.float32, device="cuda")
-    with pytest.raises(ValueError, match="scales must be contiguous"):
+    with pytest.raises(ValueError, match="non-contiguous scales view"):
         pqg.quant(x, out, tall[:, ::2], group=128, scale_fmt="fp32", layout="col")
+    # a transposed column-major plane of the right size is not a row-major one
+    with pytest.raises(ValueError, match="layout 'row' does not match"):
+        pqg.quant(x, out, sc.transpose(-1, -2), group=128, scale_fmt="fp32", layout="row")
     xe = torch.randn(4, M, K, device="cuda").to(torch.bfloat16)
     counts = torch.full((8,), M, dtype=torch.int32, device="cuda")
     with pytest.raises(ValueError, match="masked_m must be a contiguous"):
@@ -313,6 +313,21 @@ def test_torch_helper_rejects_strided_buffers():
     torch.cuda.synchronize()
     assert torch.equal(q.view(torch.uint8), q2.view(torch.uint8))
     assert torch.equal(sc, s2)
+
+
+@pytest.mark.skipif(torch.cuda.device_count() < 2, reason="needs two CUDA devices")
+def test_torch_helper_runs_on_the_tensors_device():
+    """quant() makes x's device current for the call: with another device
+    current, the codes still match those of a call on x's own device."""
+    M, K = 256, 2048
+    x = torch.randn(M, K, device="cuda:1").to(torch.bfloat16)
+    with torch.cuda.device(0):
+        q, s = pqg.quant(x, group=128, scale_fmt="ue8m0", layout="packed")
+    with torch.cuda.device(1):
+        q2, s2 = pqg.quant(x, group=128, scale_fmt="ue8m0", layout="packed")
+        torch.cuda.synchronize()
+    assert q.device == x.device
+    assert torch.equal(q.view(torch.uint8), q2.view(torch.uint8)) and torch.equal(s, s2)
 
 
 # --------------------------------------------------------------------------

@@ -172,6 +172,17 @@ def max_over_ranks(value: float, device, world: int) -> float:
     return float(t.item())
 
 
+def max_over_ranks_all(values, device, world: int):
+    """Element-wise max over ranks of a list of per-sample times."""
+    if world <= 1:
+        return list(values)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
 def job_throughput(bytes_per_step: int, steps: int, ms: float, world: int) -> float:
     """Whole-job GB/s: every rank's bytes over the slowest rank's interval."""
     return world * bytes_per_step * steps / (ms * 1e-3) / 1e9
@@ -372,8 +383,10 @@ def run_ours(args, w, rank: int, world: int, local_rank: int) -> dict | None:
         # of the timed region); warm-up steps run eagerly before capture
         stream = torch.cuda.Stream(dev)
         sh = stream.cuda_stream
+    t_host = time.perf_counter()
     for i in range(args.warmup):
         launch(i)
+    host_us = (time.perf_counter() - t_host) * 1e6 / max(args.warmup, 1)
     if args.graph:
         torch.cuda.synchronize(dev)
         graph = torch.cuda.CUDAGraph()
@@ -382,35 +395,64 @@ def run_ours(args, w, rank: int, world: int, local_rank: int) -> dict | None:
             for i in range(args.steps):
                 launch(args.warmup + i)
         captured = pqg.pqg_launch_count() - captured0
-    barrier()
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    # Each sample times exactly K steps between a barrier + synchronize on
+    # both sides.  Stream launches are queued behind a short device-side sleep
+    # issued before the start event, so that the host's launch cost is not
+    # inside the timed interval (the sleep covers the time the host needs to
+    # queue the K launches).
+    sleep_cycles = int(min(1.5 * args.steps * host_us + 20.0, 50e3) * 2e3)   # ~2 GHz
+
+    def sample():
+        barrier()
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            if graph is None:
+                torch.cuda._sleep(sleep_cycles)
+            start.record(stream)
+            if graph is not None:
+                # replay on the capture stream, where the events are recorded
+                graph.replay()
+            else:
+                for i in range(args.steps):
+                    launch(args.warmup + i)
+            end.record(stream)
+        end.synchronize()
+        barrier()
+        return start.elapsed_time(end)
+
     launches0 = pqg.pqg_launch_count()
     with ClockSampler(dev.index) as clocks:
-        start.record(stream)
-        if graph is not None:
-            # replay on the capture stream: torch replays on the current stream,
-            # and the events are recorded on `stream`
-            with torch.cuda.stream(stream):
-                graph.replay()
-        else:
-            for i in range(args.steps):
-                launch(args.warmup + i)
-        end.record(stream)
-        end.synchronize()
-    barrier()
-    launches = captured if graph is not None else pqg.pqg_launch_count() - launches0
+        first = max_over_ranks(sample(), dev, world)
+        # at least 10 samples and at least ~100 ms of timed GPU work in total
+        n_samples = args.samples or int(min(max(10, -(-100.0 // max(first, 1e-3))), 2000))
+        times = [sample() for _ in range(n_samples - 1)]
+    launches = (captured if graph is not None
+                else (pqg.pqg_launch_count() - launches0) // n_samples)
     del graph
-    ms = max_over_ranks(start.elapsed_time(end), dev, world)
+    per_sample = max_over_ranks_all([first] + times, dev, world)
+    ms = statistics.median(per_sample)
     ms_step = ms / args.steps
     bytes_step = w.algorithmic_bytes()
     value = job_throughput(bytes_step, args.steps, ms, world)
+    timing = {"samples": n_samples, "steps_per_sample": args.steps,
+              "ms_per_sample": {"median": ms, "min": min(per_sample), "max": max(per_sample)},
+              "value_min": job_throughput(bytes_step, args.steps, max(per_sample), world),
+              "value_max": job_throughput(bytes_step, args.steps, min(per_sample), world),
+              "method": ("each sample is the K timed steps between a barrier + synchronize on "
+                         "both sides, timed with CUDA events on the launching stream "
+                         + ("(one CUDA-graph replay)" if args.graph else
+                            "(launches queued behind a device-side sleep issued before the "
+                            "start event)")
+                         + "; value = median sample, max over ranks per sample")}
 
     lat = e2e = None
     if not args.kernel_only:
         # latency at M = 1 (same configuration, one row)
-        lat = latency_m1(w, dev, stream) if rank == 0 else None
+        lat = latency_m1(w, dev) if rank == 0 else None
         # end to end: pinned host input -> device -> quantize -> codes/scales back
         e2e = end_to_end(args, w, dev, stream, x0, outs[0], scs[0], call, world)
+    small_m = (latency_table(dev) if rank == 0 and w.name.startswith("sweep")
+               and not args.kernel_only else None)
 
     del xs, outs, scs
     torch.cuda.empty_cache()
@@ -442,25 +484,33 @@ def run_ours(args, w, rank: int, world: int, local_rank: int) -> dict | None:
         "e2e": e2e,
         "gpu_launches": launches,
         "clocks": clocks.summary(),
+        "timing": timing,
     }
+    if w.name.startswith("sweep") and not args.kernel_only:
+        line["us_per_call_small_m"] = {
+            "K": 4096, "scales": "fp32 row-major", "rows": small_m,
+            "note": "graph = 200 launches in a CUDA graph, device time per call; stream = 200 "
+                    "back-to-back launches from Python"}
     if world == 1 and not args.no_cpu_baseline and not args.kernel_only:
         line["cpu_baseline"] = cpu_baseline(w)
     return line
 
 
-def latency_m1(w, dev, stream) -> dict:
-    """µs per call at M = 1 (one row of the workload's shape and variant)."""
+def latency(w, dev, M: int = 1) -> dict:
+    """µs per call of ``w``'s variant on M rows: CUDA-graph replays (device time
+    per call) and back-to-back stream launches from Python."""
     import torch
     from precision_activation_quantization_b200 import pqg
     width = 2 * w.K if w.fused else w.K
-    x = torch.zeros((1, width), dtype=torch.bfloat16 if w.in_dtype == "bf16" else torch.float16,
+    x = torch.zeros((M, width), dtype=torch.bfloat16 if w.in_dtype == "bf16" else torch.float16,
                     device=dev)
     x.normal_()
-    out = torch.empty(w.K // 2 if w.out_dtype == "e2m1" else w.K, dtype=torch.uint8, device=dev)
-    nb = pqg.pqg_scales_bytes(1, 1, w.K, w.group, pqg.SCALE_FMTS[w.scale_fmt],
+    out = torch.empty(M * (w.K // 2 if w.out_dtype == "e2m1" else w.K), dtype=torch.uint8,
+                      device=dev)
+    nb = pqg.pqg_scales_bytes(1, M, w.K, w.group, pqg.SCALE_FMTS[w.scale_fmt],
                               pqg.LAYOUTS[w.layout])
     sc = torch.empty(nb, dtype=torch.uint8, device=dev)
-    call = make_call(w, dev, M=1)
+    call = make_call(w, dev, M=M)
     a = (x.data_ptr(), out.data_ptr(), sc.data_ptr())
     s = torch.cuda.Stream(dev)
     with torch.cuda.stream(s):
@@ -488,9 +538,33 @@ def latency_m1(w, dev, stream) -> dict:
         e1.synchronize()
         stream_us = e0.elapsed_time(e1) * 1e3 / n
     del g
-    return {"graph": graph_us, "stream": stream_us,
-            "note": "1 x K row, same variant; graph = 200 launches captured in a CUDA graph "
-                    "(device time per call); stream = 200 back-to-back launches from Python"}
+    return {"graph": graph_us, "stream": stream_us}
+
+
+def latency_m1(w, dev) -> dict:
+    """µs per call at M = 1 (one row of the workload's shape and variant)."""
+    return dict(latency(w, dev, 1),
+                note="1 x K row, same variant; graph = 200 launches captured in a CUDA graph "
+                     "(device time per call); stream = 200 back-to-back launches from Python")
+
+
+SMALL_M = (1, 16, 128, 1024)
+
+
+def latency_table(dev) -> list:
+    """µs per call of the dtype/size sweep's variants (bf16 and fp16, G = 32, 64
+    and 128, INT8 and E4M3 codes with fp32 row-major scales, K = 4096) at the
+    small row counts, where a call is latency-bound."""
+    from precision_activation_quantization_b200 import inputs
+    rows = []
+    for in_dtype in ("bf16", "fp16"):
+        for G in (32, 64, 128):
+            for out_dtype in ("int8", "e4m3"):
+                w = inputs.sweep(1, in_dtype=in_dtype, group=G, out_dtype=out_dtype)
+                for M in SMALL_M:
+                    rows.append(dict(in_dtype=in_dtype, group=G, out_dtype=out_dtype, M=M,
+                                     **latency(w, dev, M)))
+    return rows
 
 
 def end_to_end(args, w, dev, stream, x_dev, out_dev, sc_dev, call, world) -> dict:
@@ -572,6 +646,8 @@ def main():
     ap.add_argument("--workload", default="flat_hidden", choices=sorted(workloads()))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--samples", type=int, default=0,
+                    help="timed samples of K steps each (default: at least 10 and ~100 ms)")
     ap.add_argument("--graph", action="store_true",
                     help="replay the K timed steps from one CUDA graph (launch-bound workloads)")
     ap.add_argument("--kernel-only", action="store_true",

@@ -31,7 +31,10 @@ def _worker(rank, world, port, q):
     try:
         ms = 10.0 + 5.0 * rank               # rank 1 is the slow one
         got = bench.max_over_ranks(ms, torch.device("cpu"), world)
-        q.put((rank, got, bench.job_throughput(1_000_000, 100, got, world)))
+        # per-sample maxima: each rank is the slow one on some samples
+        samples = [1.0, 2.0, 3.0] if rank == 0 else [3.0, 1.0, 2.5]
+        per = bench.max_over_ranks_all(samples, torch.device("cpu"), world)
+        q.put((rank, got, bench.job_throughput(1_000_000, 100, got, world), per))
     finally:
         dist.destroy_process_group()
 
@@ -48,6 +51,7 @@ def test_max_over_ranks_and_job_throughput_gloo():
         p.join(timeout=60)
         assert p.exitcode == 0
     assert [r[1] for r in res] == [15.0, 15.0]
+    assert [r[3] for r in res] == [[3.0, 2.0, 3.0]] * 2
     # 2 ranks x 100 steps x 1 MB over 15 ms
     assert abs(res[0][2] - 2 * 100 * 1e6 / 15e-3 / 1e9) < 1e-9
 
@@ -55,6 +59,7 @@ def test_max_over_ranks_and_job_throughput_gloo():
 def test_single_rank_needs_no_process_group():
     import bench
     assert bench.max_over_ranks(3.5, None, 1) == 3.5
+    assert bench.max_over_ranks_all([3.5, 1.0], None, 1) == [3.5, 1.0]
     assert abs(bench.job_throughput(176_619_520, 1, 0.027, 1) - 6541.46) < 0.01
 
 

@@ -13,7 +13,8 @@ Source: sglang PR #30924 report, "[JIT] Trait-driven per_token_group_quant"
 (实现拆解 items 1-2; 关键源码片段 ``ref_fp8_ue8m0``; 风险与影响 on the INT8
 path), the TeleFuser "tf-kernel 安装与使用" page (使用示例, silu_and_mul halves)
 and "FlashInfer GEMM 学习笔记" §6-7 (packed TMA-aligned scales, masked_m /
-expected_m, MXFP4 at block 32 and NVFP4 at block 16).
+expected_m, MXFP4 at block 32 and NVFP4 at block 16; packed tokens per segment
+for the grouped-contiguous dispatch).
 """
 from __future__ import annotations
 
@@ -103,6 +104,14 @@ def load(path: str | None = None):
         lib.pqgo_e4m3_decode_n.argtypes = [vp, vp, i64]
         lib.pqgo_nvfp4_block_scale_n.argtypes = [vp, vp, i64, f32]
         lib.pqgo_nvfp4_multiplier_n.argtypes = [vp, vp, i64, f32]
+        lib.pqgo_varlen_rows.restype = None
+        lib.pqgo_varlen_rows.argtypes = [vp, vp, i64, i64, vp]
+        lib.pqgo_quant_varlen.restype = i32
+        lib.pqgo_quant_varlen.argtypes = [vp, vp, vp, i64, i64, i32, i32, i32, i32, i32, i32,
+                                          vp, vp, i64]
+        lib.pqgo_quant_varlen_nvfp4.restype = i32
+        lib.pqgo_quant_varlen_nvfp4.argtypes = [vp, vp, vp, i64, i64, i32, i32, i32, vp, vp,
+                                                i64, f32]
         if default:
             _lib = lib
         return lib
@@ -283,6 +292,69 @@ def quant(x_bits, *, M: int, K: int, group: int, E: int = 1, in_dtype: str = "bf
                         int(in_dtype == "fp16"), OUT_KINDS[out_dtype],
                         int(scale_fmt == "ue8m0"), LAYOUTS[layout], int(bool(fused)),
                         None if mm is None else _ptr(mm))
+    if rc != 0:
+        raise ValueError(f"oracle rejected the call (status {rc})")
+    return out, scales
+
+
+# --------------------------------------------------------------------------
+# grouped-contiguous (varlen) dispatch
+# --------------------------------------------------------------------------
+
+def varlen_rows(seg_indptr, seg_lens, M: int, lib=None) -> np.ndarray:
+    """bool [M]: the token rows of the segments (see pqgo_varlen_rows)."""
+    lib = lib or load()
+    ip = _c(seg_indptr, np.int32)
+    E = ip.size - 1
+    ln = None if seg_lens is None else _c(seg_lens, np.int32)
+    if E < 1 or (ln is not None and ln.size != E):
+        raise ValueError("seg_indptr needs E + 1 entries and seg_lens E")
+    live = np.empty(max(M, 1), np.uint8)
+    lib.pqgo_varlen_rows(_ptr(ip), None if ln is None else _ptr(ln), E, M, _ptr(live))
+    return live[:M].astype(bool)
+
+
+def quant_varlen(x_bits, *, M: int, K: int, group: int, seg_indptr, seg_lens=None,
+                 in_dtype: str = "bf16", out_dtype: str = "e4m3", scale_fmt: str = "fp32",
+                 layout: str = "row", fused: bool = False, out: np.ndarray | None = None,
+                 scales: np.ndarray | None = None, fill: int = 0xA5, global_scale=None,
+                 lib=None):
+    """Grouped-contiguous (varlen) call on M packed rows ([M, K], [M, 2K] fused):
+    only the token rows of the segments are quantized, into the same rows of
+    ``out`` and of one scale plane of M rows.  Returns (out [M, K] or [M, K/2],
+    scales shaped as a flat call's [1, ...]); untouched bytes keep ``fill``."""
+    lib = lib or load()
+    x = _c(x_bits, np.uint16)
+    width = 2 * K if fused else K
+    if x.size != M * width:
+        raise ValueError(f"x has {x.size} elements, expected {M * width}")
+    ip = _c(seg_indptr, np.int32)
+    E = ip.size - 1
+    ln = None if seg_lens is None else _c(seg_lens, np.int32)
+    if E < 1 or (ln is not None and ln.size != E):
+        raise ValueError("seg_indptr needs E + 1 entries and seg_lens E")
+    kbytes = K // 2 if out_dtype == "e2m1" else K
+    if out is None:
+        out = np.full((M, kbytes), fill, np.uint8)
+    shape, sdt = scales_shape(1, M, K, group, scale_fmt, layout)
+    if scales is None:
+        scales = np.empty(shape, sdt)
+        scales.view(np.uint8).fill(fill)
+    nbytes = lib.pqgo_scales_nbytes(1, M, K, group, int(scale_fmt != "fp32"), LAYOUTS[layout])
+    if scales.nbytes != nbytes or out.size != M * kbytes:
+        raise ValueError("output buffers have the wrong size")
+    lp = None if ln is None else _ptr(ln)
+    if scale_fmt == "e4m3":
+        if out_dtype != "e2m1" or group != 16 or global_scale is None:
+            raise ValueError("E4M3 block scales are NVFP4: e2m1 codes, group 16, a global scale")
+        rc = lib.pqgo_quant_varlen_nvfp4(_ptr(x), _ptr(out), _ptr(scales), M, K,
+                                         int(in_dtype == "fp16"), LAYOUTS[layout],
+                                         int(bool(fused)), _ptr(ip), lp, E, float(global_scale))
+    else:
+        rc = lib.pqgo_quant_varlen(_ptr(x), _ptr(out), _ptr(scales), M, K, group,
+                                   int(in_dtype == "fp16"), OUT_KINDS[out_dtype],
+                                   int(scale_fmt == "ue8m0"), LAYOUTS[layout], int(bool(fused)),
+                                   _ptr(ip), lp, E)
     if rc != 0:
         raise ValueError(f"oracle rejected the call (status {rc})")
     return out, scales

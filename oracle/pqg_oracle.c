@@ -58,6 +58,16 @@
  *     inside a tile the exponent of (row m, group g) at byte
  *     (m % 32) * 16 + ((m / 32) % 4) * 4 + (g % 4).  Bytes of padding columns
  *     (groups >= ng) in a quantized row are 0; padding rows are not written.
+ *   - grouped-contiguous (varlen) dispatch ([PR] 实现拆解 item 4, the varlen
+ *     DeepGEMM caller quantizing through per_token_group_quant; [FI] section 7,
+ *     packed tokens of all experts in one buffer, mapped per segment by
+ *     seg_indptr / seg_lens): M packed rows hold E segments; segment e spans
+ *     rows [indptr[e], indptr[e+1]) (both ends clamped into [0, M], the end no
+ *     lower than the start), and its first lens[e] rows (clamped into the
+ *     segment; every row when lens is absent) are tokens, the rest padding.
+ *     Token rows are quantized exactly as in a flat call over the M rows, with
+ *     codes and scales at the same row of one scale plane of M rows; padding
+ *     rows are not touched.
  *
  * Build: gcc -O2 -std=c11 -fPIC -shared -ffp-contract=off (no fast-math).
  * Floating point: C float arithmetic is IEEE binary32 with round-to-nearest
@@ -291,10 +301,10 @@ int64_t pqgo_scales_nbytes(int64_t E, int64_t M, int64_t K, int G,
  *   masked_m: host array of E row counts, or NULL.  Rows m >= masked_m[e]
  *             (clamped to [0, M]) are not touched; neither are padding rows.
  * Returns 0, -1 for an invalid argument, -2 for a non-finite input value. */
-int pqgo_quant(const uint16_t *in, uint8_t *out, void *scales, int64_t E,
-               int64_t M, int64_t K, int G, int in_fp16, int out_kind,
-               int scale_ue8m0, int layout, int fused,
-               const int32_t *masked_m) {
+static int quant_rows(const uint16_t *in, uint8_t *out, void *scales, int64_t E,
+                      int64_t M, int64_t K, int G, int in_fp16, int out_kind,
+                      int scale_ue8m0, int layout, int fused,
+                      const int32_t *masked_m, const uint8_t *row_live) {
     const int out_int8 = out_kind == PQGO_OUT_INT8;
     const int out_e2m1 = out_kind == PQGO_OUT_E2M1;
     if (E < 1 || M < 0 || K <= 0 || G <= 0 || K % G != 0) return -1;
@@ -319,6 +329,7 @@ int pqgo_quant(const uint16_t *in, uint8_t *out, void *scales, int64_t E,
             if (rows > M) rows = M;
         }
         for (int64_t m = 0; m < rows && status == 0; ++m) {
+            if (row_live && !row_live[m]) continue;   /* varlen padding row */
             const uint16_t *xrow = in + (e * M + m) * in_width;
             uint8_t *qrow = out + (e * M + m) * (out_e2m1 ? K / 2 : K);
             for (int64_t g = 0; g < ng; ++g) {
@@ -400,6 +411,14 @@ int pqgo_quant(const uint16_t *in, uint8_t *out, void *scales, int64_t E,
     return status;
 }
 
+int pqgo_quant(const uint16_t *in, uint8_t *out, void *scales, int64_t E,
+               int64_t M, int64_t K, int G, int in_fp16, int out_kind,
+               int scale_ue8m0, int layout, int fused,
+               const int32_t *masked_m) {
+    return quant_rows(in, out, scales, E, M, K, G, in_fp16, out_kind, scale_ue8m0, layout,
+                      fused, masked_m, NULL);
+}
+
 /* NVFP4 quantization of E experts of M rows of K outputs (K a multiple of 16).
  *   in, masked_m, fused: as for pqgo_quant.
  *   out    : [E][M][K/2] bytes of E2M1 code pairs (element 2i in bits 0-3).
@@ -407,9 +426,9 @@ int pqgo_quant(const uint16_t *in, uint8_t *out, void *scales, int64_t E,
  *            PQGO_COL ([E][K/16][M_pad]) or PQGO_TILE128X4 (as for MXFP4).
  *   g      : the global scale (finite, > 0).
  * Returns 0, -1 for an invalid argument, -2 for a non-finite input value. */
-int pqgo_quant_nvfp4(const uint16_t *in, uint8_t *out, uint8_t *scales, int64_t E,
-                     int64_t M, int64_t K, int in_fp16, int layout, int fused,
-                     const int32_t *masked_m, float g) {
+static int quant_rows_nvfp4(const uint16_t *in, uint8_t *out, uint8_t *scales, int64_t E,
+                            int64_t M, int64_t K, int in_fp16, int layout, int fused,
+                            const int32_t *masked_m, float g, const uint8_t *row_live) {
     const int G = PQGO_NVFP4_BLOCK;
     if (E < 1 || M < 0 || K <= 0 || K % G != 0) return -1;
     if (layout != PQGO_ROW && layout != PQGO_COL && layout != PQGO_TILE128X4) return -1;
@@ -429,6 +448,7 @@ int pqgo_quant_nvfp4(const uint16_t *in, uint8_t *out, uint8_t *scales, int64_t 
             if (rows > M) rows = M;
         }
         for (int64_t m = 0; m < rows; ++m) {
+            if (row_live && !row_live[m]) continue;   /* varlen padding row */
             const uint16_t *xrow = in + (e * M + m) * in_width;
             uint8_t *qrow = out + (e * M + m) * (K / 2);
             for (int64_t b = 0; b < ng; ++b) {
@@ -467,6 +487,74 @@ int pqgo_quant_nvfp4(const uint16_t *in, uint8_t *out, uint8_t *scales, int64_t 
         }
     }
     return 0;
+}
+
+int pqgo_quant_nvfp4(const uint16_t *in, uint8_t *out, uint8_t *scales, int64_t E,
+                     int64_t M, int64_t K, int in_fp16, int layout, int fused,
+                     const int32_t *masked_m, float g) {
+    return quant_rows_nvfp4(in, out, scales, E, M, K, in_fp16, layout, fused, masked_m, g,
+                            NULL);
+}
+
+/* ------------------------------------------------------------------------ */
+/* Grouped-contiguous (varlen) dispatch  ([PR] 实现拆解 item 4; [FI] section 7; */
+/* the reading is in the header comment)                                     */
+/* ------------------------------------------------------------------------ */
+
+/* Mark the token rows of E segments of M packed rows: row_live[r] = 1 for a
+ * token row, 0 for every other row.  Segment e spans rows [indptr[e],
+ * indptr[e+1]) with both ends clamped into [0, M] and the end no lower than
+ * the start; its first lens[e] rows, clamped into [0, segment rows], are
+ * tokens (every row of the segment when lens is NULL). */
+void pqgo_varlen_rows(const int32_t *indptr, const int32_t *lens, int64_t E, int64_t M,
+                      uint8_t *row_live) {
+    memset(row_live, 0, (size_t)M);
+    for (int64_t e = 0; e < E; ++e) {
+        int64_t start = indptr[e], end = indptr[e + 1];
+        if (start < 0) start = 0;
+        if (start > M) start = M;
+        if (end < start) end = start;
+        if (end > M) end = M;
+        int64_t n = end - start;
+        if (lens) {
+            n = lens[e];
+            if (n < 0) n = 0;
+            if (n > end - start) n = end - start;
+        }
+        for (int64_t r = start; r < start + n; ++r) row_live[r] = 1;
+    }
+}
+
+/* Quantize the token rows of M packed rows [M][K] ([M][2K] fused) in E
+ * segments (indptr: E + 1 row offsets; lens: E token counts or NULL).  Codes go
+ * to the same rows of out ([M][K], or [M][K/2] for E2M1); scales to one plane
+ * of M rows in the chosen layout (pqgo_scales_nbytes(1, M, ...) bytes).  Padding
+ * rows are not touched.  Same kinds and status values as pqgo_quant. */
+int pqgo_quant_varlen(const uint16_t *in, uint8_t *out, void *scales, int64_t M, int64_t K,
+                      int G, int in_fp16, int out_kind, int scale_ue8m0, int layout,
+                      int fused, const int32_t *indptr, const int32_t *lens, int64_t E) {
+    if (E < 1 || M < 0 || indptr == NULL) return -1;
+    uint8_t *live = (uint8_t *)malloc((size_t)(M > 0 ? M : 1));
+    if (!live) return -1;
+    pqgo_varlen_rows(indptr, lens, E, M, live);
+    int status = quant_rows(in, out, scales, 1, M, K, G, in_fp16, out_kind, scale_ue8m0,
+                            layout, fused, NULL, live);
+    free(live);
+    return status;
+}
+
+/* NVFP4 form of pqgo_quant_varlen (global scale g; layouts as pqgo_quant_nvfp4). */
+int pqgo_quant_varlen_nvfp4(const uint16_t *in, uint8_t *out, uint8_t *scales, int64_t M,
+                            int64_t K, int in_fp16, int layout, int fused,
+                            const int32_t *indptr, const int32_t *lens, int64_t E, float g) {
+    if (E < 1 || M < 0 || indptr == NULL) return -1;
+    uint8_t *live = (uint8_t *)malloc((size_t)(M > 0 ? M : 1));
+    if (!live) return -1;
+    pqgo_varlen_rows(indptr, lens, E, M, live);
+    int status = quant_rows_nvfp4(in, out, scales, 1, M, K, in_fp16, layout, fused, NULL, g,
+                                  live);
+    free(live);
+    return status;
 }
 
 /* ------------------------------------------------------------------------ */

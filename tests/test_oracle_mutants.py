@@ -73,6 +73,25 @@ MUTANTS = {
     "nvfp4_tile_plane_floor": ("const int64_t plane = ((M + 127) / 128) * ((ng + 3) / 4) * 512;",
                                "const int64_t plane = (M / 128) * ((ng + 3) / 4) * 512;"),
     "nvfp4_tile_padding_not_zeroed": ("scales[e * plane + tile128x4_offset(m, b, ng)] = 0;", ";"),
+    "varlen_lens_ignored": ("        if (lens) {\n            n = lens[e];",
+                            "        if (0) {\n            n = lens[e];"),
+    "varlen_lens_not_clamped_to_segment": ("if (n > end - start) n = end - start;", ";"),
+    "varlen_segment_from_next_offset": ("int64_t start = indptr[e], end = indptr[e + 1];",
+                                        "int64_t start = indptr[e + 1], end = indptr[e + 1];"),
+    "varlen_padding_rows_quantized": (
+        "if (row_live && !row_live[m]) continue;   /* varlen padding row */\n"
+        "            const uint16_t *xrow = in + (e * M + m) * in_width;\n"
+        "            uint8_t *qrow = out + (e * M + m) * (out_e2m1",
+        "if (0) continue;   /* varlen padding row */\n"
+        "            const uint16_t *xrow = in + (e * M + m) * in_width;\n"
+        "            uint8_t *qrow = out + (e * M + m) * (out_e2m1"),
+    "varlen_nvfp4_padding_rows_quantized": (
+        "if (row_live && !row_live[m]) continue;   /* varlen padding row */\n"
+        "            const uint16_t *xrow = in + (e * M + m) * in_width;\n"
+        "            uint8_t *qrow = out + (e * M + m) * (K / 2);",
+        "if (0) continue;   /* varlen padding row */\n"
+        "            const uint16_t *xrow = in + (e * M + m) * in_width;\n"
+        "            uint8_t *qrow = out + (e * M + m) * (K / 2);"),
 }
 
 

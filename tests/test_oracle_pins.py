@@ -776,6 +776,143 @@ def test_masked_tiled_planes_hold_whole_tiles(fmt):
     assert (s[1] == 0xA5).all()
 
 
+# --------------------------------------------------------------------------
+# Grouped-contiguous (varlen) dispatch: packed tokens in per-expert segments
+# --------------------------------------------------------------------------
+
+# (seg_indptr, seg_lens, M) -> token rows, each worked by hand from the rule:
+# segment e spans [indptr[e], indptr[e+1]) clamped into [0, M] (end >= start),
+# and its first lens[e] rows, clamped into the segment, are tokens.
+VARLEN_MASKS = [
+    # DeepGEMM-style: segments padded to 4 rows; 3, 0, 8 (of 9 asked) and 4 tokens
+    (([0, 4, 4, 12, 16], [3, 0, 9, 4], 16), [0, 1, 2] + list(range(4, 12)) + [12, 13, 14, 15]),
+    # no lens: every row of every segment is a token (ragged, unpadded)
+    (([0, 3, 5, 9], None, 10), list(range(9))),
+    # a negative count, a start below 0, an end past M
+    (([-2, 2, 6, 40], [5, -1, 9], 8), [0, 1, 6, 7]),
+    # a decreasing offset leaves an empty segment; the next starts at its own offset
+    (([0, 6, 3, 8], [2, 4, 3], 8), [0, 1, 3, 4, 5]),
+    # segments need not start at row 0 or cover every row
+    (([5, 7, 7], [2, 9], 9), [5, 6]),
+]
+
+
+@pytest.mark.parametrize("case,rows", VARLEN_MASKS, ids=[str(i) for i in range(len(VARLEN_MASKS))])
+def test_varlen_token_rows_by_hand(case, rows):
+    indptr, lens, M = case
+    live = oracle.varlen_rows(np.array(indptr, np.int32),
+                              None if lens is None else np.array(lens, np.int32), M)
+    assert sorted(np.flatnonzero(live).tolist()) == rows
+
+
+def _varlen_planes(row, live, layout, plane_bytes):
+    """The bytes one scale plane of M rows must hold when only the rows with
+    live[m] are quantized: the row-major byte table ``row`` [M, ng] at each
+    layout's defined position for those rows (padding groups 0), the sentinel
+    everywhere else."""
+    M, ng = row.shape
+    mpad, nw = (M + 3) // 4 * 4, (ng + 3) // 4
+    want = np.full(plane_bytes, 0xA5, np.uint8)
+    for m in np.flatnonzero(live):
+        for g in range(ng if layout in ("row", "col") else 4 * nw):
+            v = row[m, g] if g < ng else 0
+            if layout == "row":
+                want[m * ng + g] = v
+            elif layout == "col":
+                want[g * mpad + m] = v
+            elif layout == "packed":
+                want[((g // 4) * mpad + m) * 4 + g % 4] = v
+            else:
+                r = m % 128
+                want[((m // 128) * nw + g // 4) * 512 + (r % 32) * 16 + (r // 32) * 4 + g % 4] = v
+    return want
+
+
+@st.composite
+def _varlen_case(draw):
+    E = draw(st.integers(1, 5))
+    caps = draw(st.lists(st.sampled_from([0, 1, 3, 4, 8, 128]), min_size=E, max_size=E))
+    indptr = np.concatenate([[0], np.cumsum(caps)]).astype(np.int32)
+    M = int(indptr[-1]) + draw(st.sampled_from([0, 1, 5]))        # trailing rows in no segment
+    lens = (np.array([draw(st.integers(-1, c + 2)) for c in caps], np.int32)
+            if draw(st.booleans()) else None)
+    G = draw(st.sampled_from([32, 64, 128]))
+    ng = draw(st.integers(1, 6))
+    return indptr, lens, M, G, ng, draw(st.sampled_from(["bf16", "fp16"])), draw(st.integers(0, 999))
+
+
+@settings(max_examples=50, deadline=None)
+@given(_varlen_case(), st.booleans())
+def test_varlen_token_rows_are_the_flat_call_rows(case, fused):
+    """A varlen call writes, for each token row, exactly the codes and scales a
+    flat call over all M packed rows writes for that row (same row of codes,
+    same row of one scale plane of M rows, every layout), and leaves every
+    other row's codes and scale cells untouched."""
+    indptr, lens, M, G, ng, in_dtype, seed = case
+    K = ng * G
+    x = inputs.to_bits(inputs.normal((1, M, 2 * K if fused else K), seed) * 4, in_dtype)
+    live = oracle.varlen_rows(indptr, lens, M)
+    kw = dict(M=M, K=K, group=G, in_dtype=in_dtype, fused=fused)
+    for fmt, layouts in (("ue8m0", ("row", "col", "packed", "tile128x4")), ("fp32", ("row", "col"))):
+        q_flat, s_flat = oracle.quant(x, scale_fmt=fmt, layout="row", **kw)
+        q_flat = q_flat.reshape(M, K)
+        for layout in layouts:
+            q, s = oracle.quant_varlen(x, seg_indptr=indptr, seg_lens=lens, scale_fmt=fmt,
+                                       layout=layout, **kw)
+            q = q.reshape(M, K)
+            assert np.array_equal(q[live], q_flat[live])
+            assert (q[~live] == 0xA5).all()
+            if fmt == "ue8m0":
+                want = _varlen_planes(s_flat.reshape(M, ng), live, layout, s.nbytes)
+                assert np.array_equal(s.view(np.uint8).reshape(-1), want), layout
+            else:
+                f = s.view(np.uint32).reshape(-1)
+                ref = s_flat.view(np.uint32).reshape(M, ng)
+                mpad = (M + 3) // 4 * 4
+                idx = (np.arange(M)[:, None] * ng + np.arange(ng)[None, :] if layout == "row"
+                       else np.arange(ng)[None, :] * mpad + np.arange(M)[:, None])
+                assert np.array_equal(f[idx[live]], ref[live])
+                mask = np.ones(f.size, bool)
+                mask[idx[live].reshape(-1)] = False
+                assert (f[mask] == 0xA5A5A5A5).all()
+
+
+@settings(max_examples=25, deadline=None)
+@given(_varlen_case(), st.sampled_from([1.0, 2.625]), st.sampled_from(["row", "col", "tile128x4"]))
+def test_varlen_nvfp4_token_rows_are_the_flat_call_rows(case, g, layout):
+    """The same property for NVFP4 (blocks of 16, E4M3 block scales), fused."""
+    indptr, lens, M, _, ng, in_dtype, seed = case
+    K = ng * 16
+    x = inputs.to_bits(inputs.normal((1, M, 2 * K), seed) * 4, in_dtype)
+    live = oracle.varlen_rows(indptr, lens, M)
+    kw = dict(M=M, K=K, group=16, in_dtype=in_dtype, out_dtype="e2m1", scale_fmt="e4m3",
+              fused=True, global_scale=g)
+    q_flat, s_flat = oracle.quant(x, layout="row", **kw)
+    q, s = oracle.quant_varlen(x, seg_indptr=indptr, seg_lens=lens, layout=layout, **kw)
+    q, q_flat = q.reshape(M, K // 2), q_flat.reshape(M, K // 2)
+    assert np.array_equal(q[live], q_flat[live]) and (q[~live] == 0xA5).all()
+    want = _varlen_planes(s_flat.reshape(M, ng), live, layout, s.nbytes)
+    assert np.array_equal(s.view(np.uint8).reshape(-1), want)
+
+
+def test_varlen_over_padded_segments_equals_masked_dispatch():
+    """Experts padded to M_max rows and laid end to end are the masked layout:
+    with indptr = e * M_max and lens = masked_m, the varlen codes and row-major
+    scales equal those of masked dispatch over [E, M_max]."""
+    E, M, K = 4, 12, 384
+    x = inputs.bf16_bits(inputs.normal((E, M, 2 * K), 25))
+    mm = np.array([12, 0, 5, 13], np.int32)
+    indptr = (np.arange(E + 1) * M).astype(np.int32)
+    for fmt in ("ue8m0", "fp32"):
+        qm, sm = oracle.quant(x, E=E, M=M, K=K, group=128, fused=True, scale_fmt=fmt,
+                              layout="row", masked_m=mm)
+        qv, sv = oracle.quant_varlen(x.reshape(E * M, 2 * K), M=E * M, K=K, group=128,
+                                     fused=True, scale_fmt=fmt, layout="row",
+                                     seg_indptr=indptr, seg_lens=mm)
+        assert np.array_equal(qm.reshape(-1), qv.reshape(-1))
+        assert np.array_equal(sm.view(np.uint8).reshape(-1), sv.view(np.uint8).reshape(-1))
+
+
 def test_oracle_rejects_unsupported_combinations():
     x = np.zeros((1, 4, 256), np.uint16)
     with pytest.raises(ValueError):

@@ -59,6 +59,7 @@ def workloads():
         "fused_7168": lambda: inputs.fused(M=4096, K=7168),
         "masked": lambda: inputs.masked(),
         "masked_decode": lambda: inputs.masked(decode=True),
+        "varlen": lambda: inputs.varlen(),
         "sweep_65536_bf16_e4m3_g128": lambda: inputs.sweep(65536),
         "sweep_65536_fp16_int8_g32": lambda: inputs.sweep(65536, in_dtype="fp16",
                                                           out_dtype="int8", group=32),
@@ -78,6 +79,9 @@ def describe(w) -> dict:
                        "expected_m": w.expected_m}
     if w.global_scale is not None:
         d["global_scale"] = w.global_scale
+    if w.seg_indptr is not None:
+        d["varlen"] = {"segments": w.segments, "packed_rows": w.M, "tokens": w.rows,
+                       "segment_alignment_rows": 128, "expected_m": w.expected_m}
     return d
 
 
@@ -89,6 +93,22 @@ def make_call(w, dev, M=None):
     from precision_activation_quantization_b200 import pqg
     M = w.M if M is None else M
     E = w.E if M == w.M else 1
+    if w.seg_indptr is not None:
+        # varlen: the workload's segments, or one segment of all M rows
+        full = M == w.M
+        ip = torch.from_numpy(np.asarray(w.seg_indptr if full else [0, M], np.int32)).to(dev)
+        ln = (torch.from_numpy(np.asarray(w.seg_lens, np.int32)).to(dev)
+              if full and w.seg_lens is not None else None)
+        n_seg, em = ip.numel() - 1, (w.expected_m if full else 0)
+
+        def call(a, b, c, sh):
+            return pqg.pqg_quant_varlen(a, b, c, None, M, n_seg, w.K, w.group,
+                                        pqg.IN_DTYPES[w.in_dtype], pqg.OUT_DTYPES[w.out_dtype],
+                                        pqg.SCALE_FMTS[w.scale_fmt], pqg.LAYOUTS[w.layout],
+                                        int(w.fused), ip.data_ptr(),
+                                        None if ln is None else ln.data_ptr(), em, sh)
+        call.keep = (ip, ln)
+        return call
     mm = None if (w.masked_m is None or E == 1 and M != w.M) else \
         torch.from_numpy(w.masked_m).to(dev)
     mm_ptr = None if mm is None else mm.data_ptr()
@@ -293,6 +313,11 @@ def run_reference(args, w) -> dict:
 
 def _oracle_blocks(w, rows: int):
     """(expert, first row, rows) blocks covering the workload's live rows."""
+    if w.seg_indptr is not None:
+        # varlen: the token rows of each (well-formed) segment of the one buffer
+        lens = (np.diff(w.seg_indptr) if w.seg_lens is None else w.seg_lens)
+        return [(0, int(w.seg_indptr[e]) + m0, min(rows, int(lens[e]) - m0))
+                for e in range(w.segments) for m0 in range(0, int(lens[e]), rows)]
     live = [w.M if w.masked_m is None else int(np.clip(w.masked_m[e], 0, w.M))
             for e in range(w.E)]
     return [(e, m0, min(rows, live[e] - m0)) for e in range(w.E)
@@ -303,7 +328,8 @@ def _oracle_block(w, blk):
     """Run the oracle, as it stands, on one block of rows; returns its bytes."""
     import oracle
     e, m0, n = blk
-    sub = w.with_(x=w.x[e:e + 1, m0:m0 + n], M=n, E=1, masked_m=None)
+    sub = w.with_(x=w.x[e:e + 1, m0:m0 + n], M=n, E=1, masked_m=None, seg_indptr=None,
+                  seg_lens=None)
     oracle.quant(sub.x, M=n, K=w.K, group=w.group, in_dtype=w.in_dtype, out_dtype=w.out_dtype,
                  scale_fmt=w.scale_fmt, layout=w.layout, fused=w.fused,
                  global_scale=w.global_scale)

@@ -212,6 +212,56 @@ PQG_API int pqg_quant_nvfp4(const void *in, void *out, void *scales,
               const int32_t *masked_m, int64_t expected_m, pqg_stream_t stream);
 
 /*
+ * pqg_quant_varlen — grouped-contiguous (varlen) dispatch: the tokens of
+ * num_experts segments packed in one buffer of M rows, as a grouped-contiguous
+ * MoE GEMM reads them.  The sglang PR #30924 report (实现拆解 item 4) has the
+ * varlen DeepGEMM caller (_varlen_deep_gemm_silu_mul_quant) quantize through
+ * per_token_group_quant; "FlashInfer GEMM 学习笔记" section 7 describes the
+ * packed-token form (GroupedContiguous: packed tokens + m_indices; segments
+ * mapped by seg_lens / seg_indptr).  The pages give no arithmetic for the
+ * segments; this library's reading:
+ *   segment e spans rows [seg_indptr[e], seg_indptr[e+1]), both ends clamped
+ *   into [0, M] and the end no lower than the start; its first seg_lens[e]
+ *   rows, clamped into the segment (every row when seg_lens is NULL), are
+ *   tokens, and the rest is padding (a grouped-contiguous GEMM pads each
+ *   expert's segment to its M block).
+ * Token rows are quantized exactly as a flat pqg_quant call over the M rows
+ * would quantize them: codes in the same row of `out`, scales in the same row
+ * of ONE scale plane of M rows.  Padding rows, and rows in no segment, are not
+ * read and not written.  Segments that overlap write the same bytes twice.
+ *
+ * in       device, read-only.  [M][K] (or [M][2K] when fuse_silu_mul) packed
+ *          rows of in_dtype.  32-byte aligned.
+ * out      device.  [M][K] code bytes ([M][K/2] for E2M1).  16-byte aligned.
+ * scales   device.  pqg_scales_bytes(1, M, K, group, scale_fmt, scale_layout)
+ *          bytes: one plane over the M packed rows in the chosen layout.
+ * global_scale  device fp32 g when scale_fmt is PQG_SCALE_E4M3 (NVFP4: group
+ *          16, out_dtype PQG_E2M1; as in pqg_quant_nvfp4), else NULL
+ *          (PQG_ERR_INVALID_ARG otherwise).
+ * M        packed rows (M >= 0; M == 0 launches nothing).
+ * num_experts  segments, 1 ..= 4096.
+ * K, group, in_dtype, out_dtype, scale_fmt, scale_layout, fuse_silu_mul:
+ *          as for pqg_quant (and pqg_quant_nvfp4 for PQG_SCALE_E4M3).
+ * seg_indptr  device int32[num_experts + 1], 4-byte aligned; must not be NULL.
+ * seg_lens device int32[num_experts] token counts, 4-byte aligned, or NULL.
+ *          Both are read on the device after the programmatic-dependent-launch
+ *          wait, so the preceding kernel on `stream` may produce them; neither
+ *          may overlap `out` or `scales`.
+ * expected_m  a hint for the grid: the typical token count of a segment
+ *          (num_experts * expected_m tokens in all).  Results never depend on
+ *          it; <= 0 or > M means M tokens.
+ * stream   as for pqg_quant.
+ *
+ * Returns PQG_OK or a negative pqg_status with nothing launched (except
+ * PQG_ERR_CUDA).  Limits: those of pqg_quant with one expert of M rows.
+ */
+PQG_API int pqg_quant_varlen(const void *in, void *out, void *scales,
+              const float *global_scale, int64_t M, int64_t num_experts, int64_t K,
+              int group, int in_dtype, int out_dtype, int scale_fmt, int scale_layout,
+              int fuse_silu_mul, const int32_t *seg_indptr, const int32_t *seg_lens,
+              int64_t expected_m, pqg_stream_t stream);
+
+/*
  * pqg_scales_bytes — size in bytes of the scale buffer pqg_quant (or, for
  * PQG_SCALE_E4M3 with group 16, pqg_quant_nvfp4) writes for these arguments
  * (all experts, padding rows included).  Returns a negative pqg_status for
@@ -231,8 +281,8 @@ PQG_API int pqg_last_cuda_error(void);
  * later pqg_quant calls of this process.  Returns the previous setting. */
 PQG_API int pqg_set_pdl(int enable);
 
-/* Number of kernels this process has launched through pqg_quant and
- * pqg_quant_nvfp4 so far. */
+/* Number of kernels this process has launched through pqg_quant,
+ * pqg_quant_nvfp4 and pqg_quant_varlen so far. */
 PQG_API uint64_t pqg_launch_count(void);
 
 /* Library version string, e.g. "pqg 0.1.0 sm_100a". */

@@ -7,6 +7,7 @@
 // size_t accessors.  The library allocates nothing and never synchronizes.
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cstdint>
 
@@ -95,16 +96,30 @@ int sm_count(int device) {
 
 namespace {
 
-// Validation and launch shared by pqg_quant and pqg_quant_nvfp4.
+// Varlen (grouped-contiguous) segments: E + 1 row offsets and E token counts
+// (or none), all on the device.
+struct Segments {
+    const int32_t *indptr;
+    const int32_t *lens;
+};
+
+// Validation and launch shared by pqg_quant, pqg_quant_nvfp4 and
+// pqg_quant_varlen (seg.indptr != nullptr: M packed rows in num_experts
+// segments, one scale plane).
 int quant_impl(const void *in, void *out, void *scales, const float *global_scale, int64_t M,
                int64_t num_experts, int64_t K, int group, int in_dtype, int out_dtype,
                int scale_fmt, int scale_layout, int fuse_silu_mul, const int32_t *masked_m,
-               int64_t expected_m, pqg_stream_t stream) {
+               int64_t expected_m, pqg_stream_t stream, Segments seg = {nullptr, nullptr}) {
+    const bool varlen = seg.indptr != nullptr;
     if (in_dtype != PQG_BF16 && in_dtype != PQG_FP16) return PQG_ERR_INVALID_ARG;
     if (out_dtype != PQG_E4M3 && out_dtype != PQG_INT8 && out_dtype != PQG_E2M1)
         return PQG_ERR_INVALID_ARG;
+    if (varlen && (num_experts < 1 || num_experts > static_cast<int64_t>(pqg::kMaxExperts)))
+        return PQG_ERR_INVALID_ARG;
+    // a varlen call is one buffer of M rows: its geometry is that of one expert
+    const int64_t planes = varlen ? 1 : num_experts;
     int64_t plane = 0;
-    const int st = check_geometry(num_experts, M, K, group, scale_fmt, scale_layout, &plane);
+    const int st = check_geometry(planes, M, K, group, scale_fmt, scale_layout, &plane);
     if (st != PQG_OK) return st;
     const bool nvfp4 = scale_fmt == PQG_SCALE_E4M3;
     if (scale_fmt == PQG_SCALE_UE8M0 && out_dtype == PQG_INT8) return PQG_ERR_UNSUPPORTED;
@@ -122,25 +137,37 @@ int quant_impl(const void *in, void *out, void *scales, const float *global_scal
         if (!aligned(scales, 4)) return PQG_ERR_ALIGNMENT;  // word stores
     }
     if (masked_m != nullptr && !aligned(masked_m, 4)) return PQG_ERR_ALIGNMENT;
+    if (varlen && (!aligned(seg.indptr, 4) || (seg.lens != nullptr && !aligned(seg.lens, 4))))
+        return PQG_ERR_ALIGNMENT;
 
     const int64_t in_row_bytes = K * 2 * (fuse_silu_mul ? 2 : 1);
-    const int64_t in_bytes = num_experts * M * in_row_bytes;
+    const int64_t in_bytes = planes * M * in_row_bytes;
     const int64_t out_row_bytes = out_dtype == PQG_E2M1 ? K / 2 : K;
-    const int64_t out_bytes = num_experts * M * out_row_bytes;
-    if (overlaps(in, in_bytes, out, out_bytes) || overlaps(in, in_bytes, scales, plane * num_experts) ||
-        overlaps(out, out_bytes, scales, plane * num_experts))
+    const int64_t out_bytes = planes * M * out_row_bytes;
+    if (overlaps(in, in_bytes, out, out_bytes) || overlaps(in, in_bytes, scales, plane * planes) ||
+        overlaps(out, out_bytes, scales, plane * planes))
         return PQG_ERR_INVALID_ARG;
+    if (varlen) {
+        // the segment tables are read by every CTA: no output may overwrite them
+        const int64_t ib = 4 * (num_experts + 1), lb = seg.lens != nullptr ? 4 * num_experts : 0;
+        if (overlaps(seg.indptr, ib, out, out_bytes) || overlaps(seg.indptr, ib, scales, plane) ||
+            overlaps(seg.lens, lb, out, out_bytes) || overlaps(seg.lens, lb, scales, plane))
+            return PQG_ERR_INVALID_ARG;
+    }
 
     pqg::LaunchArgs a;
     a.p.in = static_cast<const uint8_t *>(in);
     a.p.out = static_cast<uint8_t *>(out);
     a.p.scales = static_cast<uint8_t *>(scales);
-    a.p.masked_m = masked_m;
+    a.p.masked_m = varlen ? nullptr : masked_m;
+    a.p.seg_indptr = seg.indptr;
+    a.p.seg_lens = seg.lens;
     a.p.gscale = global_scale;
-    a.p.in_expert_bytes = M * in_row_bytes;
-    a.p.out_expert_bytes = M * out_row_bytes;
+    // varlen segments address the one packed buffer by their own row offsets
+    a.p.in_expert_bytes = varlen ? 0 : M * in_row_bytes;
+    a.p.out_expert_bytes = varlen ? 0 : M * out_row_bytes;
     a.p.out_row_bytes = static_cast<uint32_t>(out_row_bytes);
-    a.p.scale_expert_bytes = plane;
+    a.p.scale_expert_bytes = varlen ? 0 : plane;
     a.p.M = static_cast<uint32_t>(M);
     a.p.K = static_cast<uint32_t>(K);
     a.p.in_row_bytes = static_cast<uint32_t>(in_row_bytes);
@@ -149,16 +176,24 @@ int quant_impl(const void *in, void *out, void *scales, const float *global_scal
     a.p.mpad = static_cast<uint32_t>(padded_rows(M));
     a.p.layout = static_cast<uint32_t>(scale_layout);
     a.p.experts = static_cast<uint32_t>(num_experts);
-    const int64_t grid_rows =
-        (masked_m != nullptr && expected_m > 0 && expected_m < M) ? expected_m : M;
-    a.expected_strips = static_cast<uint64_t>(num_experts * grid_rows) * a.p.segs;
-    a.expected_rows = static_cast<uint64_t>(num_experts * grid_rows);
+    // rows the grid is sized for: every expert's expected_m when masked, or
+    // (varlen) num_experts * expected_m tokens, at most the M packed rows
+    int64_t grid_total = num_experts * M;
+    if (varlen)
+        grid_total = (expected_m > 0 && expected_m <= M) ? std::min(M, num_experts * expected_m)
+                                                         : M;
+    else if (masked_m != nullptr && expected_m > 0 && expected_m < M)
+        grid_total = num_experts * expected_m;
+    if (grid_total < 1) grid_total = 1;
+    a.expected_strips = static_cast<uint64_t>(grid_total) * a.p.segs;
+    a.expected_rows = static_cast<uint64_t>(grid_total);
     a.group = group;
     a.kind = nvfp4                            ? pqg::Kind::E2M1_E4M3
              : out_dtype == PQG_E2M1          ? pqg::Kind::E2M1_UE8M0
              : scale_fmt == PQG_SCALE_UE8M0 ? pqg::Kind::E4M3_UE8M0
              : out_dtype == PQG_INT8        ? pqg::Kind::INT8_FP32
                                             : pqg::Kind::E4M3_FP32;
+    a.disp = varlen ? pqg::kVarlen : num_experts > 1 ? pqg::kMasked : pqg::kFlat;
     a.fused = fuse_silu_mul != 0;
     a.pdl = g_pdl.load(std::memory_order_relaxed) != 0;
     a.stream = reinterpret_cast<cudaStream_t>(stream);
@@ -201,6 +236,18 @@ int pqg_quant_nvfp4(const void *in, void *out, void *scales, const float *global
     return quant_impl(in, out, scales, global_scale, M, num_experts, K, 16, in_dtype, PQG_E2M1,
                       PQG_SCALE_E4M3, scale_layout, fuse_silu_mul, masked_m, expected_m,
                       stream);
+}
+
+int pqg_quant_varlen(const void *in, void *out, void *scales, const float *global_scale,
+                     int64_t M, int64_t num_experts, int64_t K, int group, int in_dtype,
+                     int out_dtype, int scale_fmt, int scale_layout, int fuse_silu_mul,
+                     const int32_t *seg_indptr, const int32_t *seg_lens, int64_t expected_m,
+                     pqg_stream_t stream) {
+    if (seg_indptr == nullptr) return PQG_ERR_INVALID_ARG;
+    if ((scale_fmt == PQG_SCALE_E4M3) != (global_scale != nullptr)) return PQG_ERR_INVALID_ARG;
+    return quant_impl(in, out, scales, global_scale, M, num_experts, K, group, in_dtype,
+                      out_dtype, scale_fmt, scale_layout, fuse_silu_mul, nullptr, expected_m,
+                      stream, Segments{seg_indptr, seg_lens});
 }
 
 const char *pqg_status_string(int status) {

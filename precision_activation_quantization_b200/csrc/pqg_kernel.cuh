@@ -19,7 +19,10 @@
 // CTAs take round-robin.  With several experts each CTA first prefix-sums the
 // per-expert strip counts (in each warp's registers up to 32 experts, in
 // shared memory beyond), so a warp can find the expert and row of any strip;
-// skewed masked_m cannot leave CTAs idle.
+// skewed masked_m cannot leave CTAs idle.  Grouped-contiguous (varlen)
+// dispatch uses the same table over the token rows of E segments of one packed
+// buffer (each segment's first row kept beside its count), so padding rows are
+// never visited.
 //
 // Memory-level parallelism.  A warp takes ITEMS strips per chunk and issues
 // all of the chunk's 32-byte loads before any arithmetic; with 32-48 resident
@@ -106,11 +109,13 @@ struct Params {
     uint8_t *out;              // expert 0, row 0
     uint8_t *scales;           // expert 0's scale plane (byte address)
     const int32_t *masked_m;   // device int32[experts], or null: all M rows
+    const int32_t *seg_indptr; // varlen: device int32[experts + 1] segment row offsets
+    const int32_t *seg_lens;   // varlen: device int32[experts] token counts, or null
     const float *gscale;       // NVFP4 only: device fp32 global scale g
     int64_t in_expert_bytes;   // M * in_row_bytes
     int64_t out_expert_bytes;  // M * out_row_bytes
     int64_t scale_expert_bytes;
-    uint32_t M;                // rows per expert (capacity when masked)
+    uint32_t M;                // rows per expert (capacity when masked; all rows when varlen)
     uint32_t K;                // outputs per row
     uint32_t in_row_bytes;     // 2K (plain) or 4K (fused), in bytes
     uint32_t out_row_bytes;    // K (one byte per code) or K/2 (E2M1, two per byte)
@@ -122,10 +127,16 @@ struct Params {
     uint32_t items;            // strips per warp per block, 1 .. ITEMS
 };
 
+// Dispatch forms: one expert's M rows (flat), E experts of M rows each with a
+// per-expert row count (masked), or E segments of one buffer of M packed rows
+// (varlen, grouped-contiguous: expert strides are 0 and a segment's rows
+// start at its own row offset).
+enum : int { kFlat = 0, kMasked = 1, kVarlen = 2 };
+
 // Dynamic shared memory of one CTA: the expert prefix table (more than 32
-// experts only).
-__host__ __device__ constexpr uint32_t smem_bytes(uint32_t experts) {
-    return experts > 32u ? 4u * (experts + 1u) : 0u;
+// experts only), followed by the segments' first rows when varlen.
+__host__ __device__ constexpr uint32_t smem_bytes(uint32_t experts, bool varlen = false) {
+    return experts > 32u ? 4u * (experts + 1u) + (varlen ? 4u * experts : 0u) : 0u;
 }
 
 // ---------------------------------------------------------------------------
@@ -487,12 +498,16 @@ __device__ __forceinline__ void encode16(const float (&v)[16], const GroupScale 
 // ---------------------------------------------------------------------------
 //
 // Strips of expert e are [start_e, start_e + strips_e); strips_e =
-// rows_e * segs with rows_e = clamp(masked_m[e], 0, M) (M without masked_m).
-// Three representations, picked per launch:
+// rows_e * segs with rows_e = clamp(masked_m[e], 0, M) (M without masked_m),
+// or, varlen, the token rows of segment e (see segment() below), whose first
+// row base_e is the segment's offset.  Three representations, picked per
+// launch:
 //   one expert   : start 0, strips = total (no table at all);
-//   <= 32 experts: a warp-register table, lane e holding expert e's count and
-//                  inclusive prefix; a lookup is one ballot and two shuffles;
-//   more experts : a shared-memory prefix table built by the CTA.
+//   <= 32 experts: a warp-register table, lane e holding expert e's count,
+//                  inclusive prefix (and first row); a lookup is one ballot and
+//                  two (three) shuffles;
+//   more experts : a shared-memory prefix table built by the CTA (followed by
+//                  the first rows).
 
 constexpr uint32_t kWarpTableExperts = 32;
 
@@ -501,31 +516,52 @@ struct ExpertTable {
     uint32_t total;    // strips of all experts
     uint32_t incl;     // mode 1: this lane's inclusive prefix (total for lanes >= E)
     uint32_t cnt;      // mode 1: this lane's expert's strips
-    const uint32_t *prefix;  // mode 2: prefix[e] = start_e, prefix[E] = total
+    uint32_t base;     // varlen, modes 0-1: first row of (this lane's) segment
+    const uint32_t *prefix;  // mode 2: prefix[e] = start_e, prefix[E] = total;
+                             // varlen: prefix[E + 1 + e] = first row of segment e
 };
 
 struct Span {
-    uint32_t e, start, strips;
+    uint32_t e, start, strips, base;   // base: first row (varlen), else 0
 };
 
-__device__ __forceinline__ uint32_t expert_strips(const Params &p, uint32_t e) {
+// Segment e of a varlen call: rows [indptr[e], indptr[e+1]) clamped into
+// [0, M] with the end no lower than the start; its first lens[e] rows,
+// clamped into the segment (all of them without lens), are tokens.
+__device__ __forceinline__ uint32_t segment_rows(const Params &p, uint32_t e, uint32_t &first) {
+    const int M = static_cast<int>(p.M);
+    const int s = min(max(__ldg(p.seg_indptr + e), 0), M);
+    const int end = min(max(__ldg(p.seg_indptr + e + 1), s), M);
+    int n = end - s;
+    if (p.seg_lens != nullptr) n = min(max(__ldg(p.seg_lens + e), 0), n);
+    first = static_cast<uint32_t>(s);
+    return static_cast<uint32_t>(n);
+}
+
+template <bool VARLEN>
+__device__ __forceinline__ uint32_t expert_strips(const Params &p, uint32_t e, uint32_t &first) {
     uint32_t rows = p.M;
-    if (p.masked_m != nullptr) {
+    first = 0;
+    if constexpr (VARLEN) {
+        rows = segment_rows(p, e, first);
+    } else if (p.masked_m != nullptr) {
         const int mm = __ldg(p.masked_m + e);
         rows = static_cast<uint32_t>(min(max(mm, 0), static_cast<int>(p.M)));
     }
     return rows * p.segs;
 }
 
-// prefix[e] = strips of experts 0..e-1.  Every thread of the CTA calls it; it
-// ends with __syncthreads.
+// prefix[e] = strips of experts 0..e-1 (varlen: and prefix[E + 1 + e] = first
+// row of segment e).  Every thread of the CTA calls it; it ends with
+// __syncthreads.
+template <bool VARLEN>
 __device__ __forceinline__ void build_prefix(const Params &p, uint32_t *prefix) {
     __shared__ uint32_t warp_sums[32];
     const uint32_t n = blockDim.x, t = threadIdx.x, lane = t & 31u, warp = t >> 5;
     const uint32_t per = (p.experts + n - 1) / n;
     const uint32_t lo = min(t * per, p.experts), hi = min(lo + per, p.experts);
-    uint32_t local = 0;
-    for (uint32_t e = lo; e < hi; ++e) local += expert_strips(p, e);
+    uint32_t local = 0, first = 0;
+    for (uint32_t e = lo; e < hi; ++e) local += expert_strips<VARLEN>(p, e, first);
     uint32_t incl = local;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -539,24 +575,26 @@ __device__ __forceinline__ void build_prefix(const Params &p, uint32_t *prefix) 
     uint32_t run = base + incl - local;
     for (uint32_t e = lo; e < hi; ++e) {
         prefix[e] = run;
-        run += expert_strips(p, e);
+        run += expert_strips<VARLEN>(p, e, first);
+        if constexpr (VARLEN) prefix[p.experts + 1u + e] = first;
     }
     if (t == n - 1) prefix[p.experts] = base + incl;
     __syncthreads();
 }
 
 // Build the table (every thread of the CTA calls it).
+template <bool VARLEN>
 __device__ __forceinline__ ExpertTable make_table(const Params &p, uint32_t *smem_prefix,
                                                   uint32_t lane) {
     ExpertTable t;
-    t.incl = t.cnt = 0;
+    t.incl = t.cnt = t.base = 0;
     t.prefix = smem_prefix;
     if (p.experts == 1) {
         t.mode = 0;
-        t.total = expert_strips(p, 0);
+        t.total = expert_strips<VARLEN>(p, 0, t.base);
     } else if (p.experts <= kWarpTableExperts) {
         t.mode = 1;
-        t.cnt = lane < p.experts ? expert_strips(p, lane) : 0u;
+        t.cnt = lane < p.experts ? expert_strips<VARLEN>(p, lane, t.base) : 0u;
         uint32_t incl = t.cnt;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
@@ -567,25 +605,29 @@ __device__ __forceinline__ ExpertTable make_table(const Params &p, uint32_t *sme
         t.total = __shfl_sync(0xFFFFFFFFu, incl, 31);
     } else {
         t.mode = 2;
-        build_prefix(p, smem_prefix);
+        build_prefix<VARLEN>(p, smem_prefix);
         t.total = smem_prefix[p.experts];
     }
     return t;
 }
 
 // The expert holding strip s (s < total).  Warp-uniform s; every lane calls.
+template <bool VARLEN>
 __device__ __forceinline__ Span locate(const ExpertTable &t, uint32_t experts, uint32_t s) {
     Span sp;
+    sp.base = 0;
     if (t.mode == 0) {
         sp.e = 0;
         sp.start = 0;
         sp.strips = t.total;
+        if constexpr (VARLEN) sp.base = t.base;
     } else if (t.mode == 1) {
         // experts whose whole range lies at or below s come first
         sp.e = __popc(__ballot_sync(0xFFFFFFFFu, t.incl <= s));
         const uint32_t incl = __shfl_sync(0xFFFFFFFFu, t.incl, sp.e);
         sp.strips = __shfl_sync(0xFFFFFFFFu, t.cnt, sp.e);
         sp.start = incl - sp.strips;
+        if constexpr (VARLEN) sp.base = __shfl_sync(0xFFFFFFFFu, t.base, sp.e);
     } else {
         uint32_t lo = 0, hi = experts;  // prefix[lo] <= s < prefix[hi]
         while (hi - lo > 1) {
@@ -595,6 +637,7 @@ __device__ __forceinline__ Span locate(const ExpertTable &t, uint32_t experts, u
         sp.e = lo;
         sp.start = t.prefix[lo];
         sp.strips = t.prefix[lo + 1] - sp.start;
+        if constexpr (VARLEN) sp.base = t.prefix[experts + 1u + lo];
     }
     return sp;
 }
@@ -612,41 +655,44 @@ struct Chunk {
 };
 
 // Issue the loads of strips [s, s + n) (n <= ITEMS).  Lanes past the end of a
-// ragged row load nothing.  With one expert (MULTI false) the strip index maps
+// ragged row load nothing.  With flat dispatch (kFlat) the strip index maps
 // to (row, strip-in-row) by one division; otherwise through the expert table.
-template <int ITEMS, bool FUSED, bool MULTI>
+template <int ITEMS, bool FUSED, int DISP>
 __device__ __forceinline__ void load_chunk(Chunk<ITEMS, FUSED> &ch, uint32_t s, uint32_t n,
                                            const ExpertTable &t, const Params &p,
                                            uint32_t lane) {
+    constexpr bool kVar = DISP == kVarlen;
     ch.n = n;
-    uint32_t e = 0, start = 0, end_e = t.total;
-    if constexpr (MULTI) {
-        const Span sp = locate(t, p.experts, s);
+    uint32_t e = 0, start = 0, end_e = t.total, base = 0;
+    if constexpr (DISP != kFlat) {
+        const Span sp = locate<kVar>(t, p.experts, s);
         e = sp.e;
         start = sp.start;
         end_e = sp.start + sp.strips;
+        base = sp.base;
     }
     uint32_t row = (s - start) / p.segs;
     uint32_t seg = (s - start) - row * p.segs;
 #pragma unroll
     for (int k = 0; k < ITEMS; ++k) {
         const bool live = static_cast<uint32_t>(k) < n;
-        if constexpr (MULTI) {
+        if constexpr (DISP != kFlat) {
             if (live && s + k >= end_e) {        // the chunk runs into the next expert
-                const Span sp = locate(t, p.experts, s + k);
+                const Span sp = locate<kVar>(t, p.experts, s + k);
                 e = sp.e;
                 start = sp.start;
                 end_e = sp.start + sp.strips;
+                base = sp.base;
                 row = 0;
                 seg = 0;
             }
         }
         ch.e[k] = e;
-        ch.row[k] = row;
+        ch.row[k] = base + row;             // varlen: the row in the packed buffer
         ch.col[k] = seg * kStripElems + lane * 16u;
         if (live && ch.col[k] < p.K) {
             const uint8_t *src = p.in + e * p.in_expert_bytes +
-                                 static_cast<uint64_t>(row) * p.in_row_bytes +
+                                 static_cast<uint64_t>(ch.row[k]) * p.in_row_bytes +
                                  static_cast<uint64_t>(ch.col[k]) * 2u;
             load32B(src, ch.x[k]);
             if constexpr (FUSED) load32B(src + static_cast<uint64_t>(p.K) * 2u, ch.u[k]);
@@ -801,16 +847,16 @@ __device__ __forceinline__ void quantize_chunk(const Chunk<ITEMS, FUSED> &ch, co
 #ifndef PQG_MIN_BLOCKS_NVFP4
 #define PQG_MIN_BLOCKS_NVFP4 6
 #endif
-template <Kind KIND, bool FUSED, bool MULTI>
+template <Kind KIND, bool FUSED, int DISP>
 constexpr int min_blocks() {
     if constexpr (FUSED) return 0;
     if constexpr (KIND == Kind::E4M3_FP32 || KIND == Kind::INT8_FP32) return PQG_MIN_BLOCKS_FP32;
-    if constexpr (KIND == Kind::E2M1_E4M3 && !MULTI) return PQG_MIN_BLOCKS_NVFP4;
+    if constexpr (KIND == Kind::E2M1_E4M3 && DISP == kFlat) return PQG_MIN_BLOCKS_NVFP4;
     return 0;
 }
 
-template <typename In, int G, Kind KIND, bool FUSED, int ITEMS, int WARPS, bool MULTI>
-__global__ void __launch_bounds__(WARPS * 32, min_blocks<KIND, FUSED, MULTI>())
+template <typename In, int G, Kind KIND, bool FUSED, int ITEMS, int WARPS, int DISP>
+__global__ void __launch_bounds__(WARPS * 32, min_blocks<KIND, FUSED, DISP>())
     quant_kernel(const __grid_constant__ Params p) {
     static_assert((G == 32 || G == 64 || G == 128) == (KIND != Kind::E2M1_E4M3) &&
                       (G == 16) == (KIND == Kind::E2M1_E4M3),
@@ -824,10 +870,11 @@ __global__ void __launch_bounds__(WARPS * 32, min_blocks<KIND, FUSED, MULTI>())
     const uint32_t warp = threadIdx.x >> 5;
     if constexpr (KIND == Kind::E2M1_E4M3) build_nvfp4_table(p, nv);
     ExpertTable t;
-    if constexpr (MULTI) {
-        t = make_table(p, smem_prefix, lane);
+    if constexpr (DISP != kFlat) {
+        t = make_table<DISP == kVarlen>(p, smem_prefix, lane);
     } else {
-        t.total = expert_strips(p, 0);
+        uint32_t first;
+        t.total = expert_strips<false>(p, 0, first);
     }
 
     // Block-cyclic schedule: a block is WARPS x items consecutive strips, CTA
@@ -841,7 +888,7 @@ __global__ void __launch_bounds__(WARPS * 32, min_blocks<KIND, FUSED, MULTI>())
         const uint32_t s = blk * block + warp * items;
         if (s >= t.total) break;                // warp-uniform
         Chunk<ITEMS, FUSED> ch;
-        load_chunk<ITEMS, FUSED, MULTI>(ch, s, min(items, t.total - s), t, p, lane);
+        load_chunk<ITEMS, FUSED, DISP>(ch, s, min(items, t.total - s), t, p, lane);
         quantize_chunk<In, G, KIND, FUSED, ITEMS>(ch, p, lane, nv);
     }
     release_dependents();

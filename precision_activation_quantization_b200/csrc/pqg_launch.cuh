@@ -22,6 +22,7 @@ struct LaunchArgs {
     uint64_t expected_rows;    // rows the grid is sized for (per-token kernel)
     int group;                 // 32 / 64 / 128, or K (per-token)
     Kind kind;
+    int disp;                  // kFlat, kMasked or kVarlen
     bool fused;
     bool pdl;
     cudaStream_t stream;
@@ -72,7 +73,7 @@ int sm_count(int device);  // cached cudaDevAttrMultiProcessorCount
 #define PQG_ITEMS_MXFP4 3
 #endif
 template <typename In, Kind KIND, int G, bool FUSED, bool MULTI>
-struct Shape {
+struct Shape {   // MULTI: several experts (masked or varlen dispatch)
     static constexpr bool kMx32 = KIND == Kind::E2M1_UE8M0 && G == 32 &&
                                   std::is_same<In, __nv_bfloat16>::value;
     static constexpr int kItems = FUSED ? (MULTI ? PQG_ITEMS_FUSED_MULTI : PQG_ITEMS_FUSED)
@@ -103,28 +104,30 @@ inline uint64_t grid_waves(uint64_t blocks, uint64_t wave) {
 
 // ITEMS_SEL > 0 overrides the variant's strips per chunk (the long flat fused
 // calls, see launch_kind).
-template <typename In, int G, Kind KIND, bool FUSED, bool MULTI, int ITEMS_SEL = 0>
+template <typename In, int G, Kind KIND, bool FUSED, int DISP, int ITEMS_SEL = 0>
 cudaError_t launch_variant(const LaunchArgs &a) {
-    using Sh = Shape<In, KIND, G, FUSED, MULTI>;
+    using Sh = Shape<In, KIND, G, FUSED, DISP != kFlat>;
     constexpr int kItems = ITEMS_SEL > 0 ? ITEMS_SEL : Sh::kItems;
     constexpr int kWarps = Sh::kWarps;
     constexpr int kThreads = kWarps * 32;
-    auto kernel = quant_kernel<In, G, KIND, FUSED, kItems, kWarps, MULTI>;
+    constexpr bool kVar = DISP == kVarlen;
+    auto kernel = quant_kernel<In, G, KIND, FUSED, kItems, kWarps, DISP>;
 
     // Resident CTAs per SM, queried once per variant without and with the
     // largest shared-memory expert table (more than 32 experts).
     static const int2 occupancy = [&] {
         int n0 = 0, n1 = 0;
         if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(smem_bytes(kMaxExperts))) != cudaSuccess ||
+                                 static_cast<int>(smem_bytes(kMaxExperts, kVar))) != cudaSuccess ||
             cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n0, kernel, kThreads, 0) !=
                 cudaSuccess ||
             cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n1, kernel, kThreads,
-                                                          smem_bytes(kMaxExperts)) != cudaSuccess)
+                                                          smem_bytes(kMaxExperts, kVar)) !=
+                cudaSuccess)
             n0 = n1 = 1;
         return make_int2(n0 < 1 ? 1 : n0, n1 < 1 ? 1 : n1);
     }();
-    const int blocks_per_sm = smem_bytes(a.p.experts) == 0 ? occupancy.x : occupancy.y;
+    const int blocks_per_sm = smem_bytes(a.p.experts, kVar) == 0 ? occupancy.x : occupancy.y;
 
     int device = 0;
     cudaError_t err = cudaGetDevice(&device);
@@ -150,7 +153,7 @@ cudaError_t launch_variant(const LaunchArgs &a) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(ctas), 1, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
-    cfg.dynamicSmemBytes = smem_bytes(a.p.experts);
+    cfg.dynamicSmemBytes = smem_bytes(a.p.experts, kVar);
     cfg.stream = a.stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -162,9 +165,12 @@ cudaError_t launch_variant(const LaunchArgs &a) {
 
 template <typename In, int G, Kind KIND>
 cudaError_t launch_kind(const LaunchArgs &a) {
+    if (a.disp == kVarlen)
+        return a.fused ? launch_variant<In, G, KIND, true, kVarlen>(a)
+                       : launch_variant<In, G, KIND, false, kVarlen>(a);
     const bool multi = a.p.experts > 1;
     if (a.fused) {
-        if (multi) return launch_variant<In, G, KIND, true, true>(a);
+        if (multi) return launch_variant<In, G, KIND, true, kMasked>(a);
         // A long flat fused call (4 or more waves of 1-strip work at 48 warps
         // per SM) runs a variant compiled for 2 strips per chunk: [4096, 2 x
         // 7168] 26.4 -> 24.6 us.  Short calls keep the 1-strip variant, whose
@@ -174,11 +180,11 @@ cudaError_t launch_kind(const LaunchArgs &a) {
         cudaError_t err = cudaGetDevice(&device);
         if (err != cudaSuccess) return err;
         const uint64_t long_call = 4ull * static_cast<uint64_t>(sm_count(device)) * 48u;
-        return a.expected_strips >= long_call ? launch_variant<In, G, KIND, true, false, 2>(a)
-                                              : launch_variant<In, G, KIND, true, false>(a);
+        return a.expected_strips >= long_call ? launch_variant<In, G, KIND, true, kFlat, 2>(a)
+                                              : launch_variant<In, G, KIND, true, kFlat>(a);
     }
-    return multi ? launch_variant<In, G, KIND, false, true>(a)
-                 : launch_variant<In, G, KIND, false, false>(a);
+    return multi ? launch_variant<In, G, KIND, false, kMasked>(a)
+                 : launch_variant<In, G, KIND, false, kFlat>(a);
 }
 
 template <typename In, int G>
@@ -223,15 +229,17 @@ inline void row_shape(uint32_t K, uint32_t *wpr, int *slots) {
     }
 }
 
-template <typename In, Kind KIND, bool FUSED, int SLOTS>
+template <typename In, Kind KIND, bool FUSED, int SLOTS, bool VARLEN>
 cudaError_t launch_row_variant(const LaunchArgs &a, uint32_t wpr) {
-    auto kernel = row_quant_kernel<In, KIND, FUSED, SLOTS>;
+    auto kernel = row_quant_kernel<In, KIND, FUSED, SLOTS, VARLEN>;
     static const int blocks_per_sm = [&] {
         int n = 0;
         if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(smem_bytes(kMaxExperts))) != cudaSuccess ||
+                                 static_cast<int>(smem_bytes(kMaxExperts, VARLEN))) !=
+                cudaSuccess ||
             cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, kRowThreads,
-                                                          smem_bytes(kMaxExperts)) != cudaSuccess ||
+                                                          smem_bytes(kMaxExperts, VARLEN)) !=
+                cudaSuccess ||
             n < 1)
             n = 1;
         return n;
@@ -252,7 +260,7 @@ cudaError_t launch_row_variant(const LaunchArgs &a, uint32_t wpr) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(ctas), 1, 1);
     cfg.blockDim = dim3(kRowThreads, 1, 1);
-    cfg.dynamicSmemBytes = smem_bytes(a.p.experts);
+    cfg.dynamicSmemBytes = smem_bytes(a.p.experts, VARLEN);
     cfg.stream = a.stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -262,16 +270,22 @@ cudaError_t launch_row_variant(const LaunchArgs &a, uint32_t wpr) {
     return cudaLaunchKernelEx(&cfg, kernel, p);
 }
 
-template <typename In, Kind KIND, bool FUSED>
-cudaError_t launch_row_kind(const LaunchArgs &a) {
+template <typename In, Kind KIND, bool FUSED, bool VARLEN>
+cudaError_t launch_row_slots(const LaunchArgs &a) {
     uint32_t wpr = 1;
     int slots = 1;
     row_shape(a.p.K, &wpr, &slots);
     switch (slots) {
-        case 1: return launch_row_variant<In, KIND, FUSED, 1>(a, wpr);
-        case 2: return launch_row_variant<In, KIND, FUSED, 2>(a, wpr);
-        default: return launch_row_variant<In, KIND, FUSED, 4>(a, wpr);
+        case 1: return launch_row_variant<In, KIND, FUSED, 1, VARLEN>(a, wpr);
+        case 2: return launch_row_variant<In, KIND, FUSED, 2, VARLEN>(a, wpr);
+        default: return launch_row_variant<In, KIND, FUSED, 4, VARLEN>(a, wpr);
     }
+}
+
+template <typename In, Kind KIND, bool FUSED>
+cudaError_t launch_row_kind(const LaunchArgs &a) {
+    return a.disp == kVarlen ? launch_row_slots<In, KIND, FUSED, true>(a)
+                             : launch_row_slots<In, KIND, FUSED, false>(a);
 }
 
 template <typename In>

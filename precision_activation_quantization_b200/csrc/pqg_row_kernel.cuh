@@ -13,8 +13,8 @@
 // iteration parity, so one barrier per row iteration is enough.  Values stay in
 // registers between the reduction and the quantization, so every input byte is
 // read once.  Rows come from the same expert table as the strip kernel
-// (counting rows instead of strips), so flat, batched and masked dispatch and
-// the fused SiLU-and-mul all work unchanged.
+// (counting rows instead of strips), so flat, batched, masked and varlen
+// dispatch and the fused SiLU-and-mul all work unchanged.
 #pragma once
 
 #include "pqg_kernel.cuh"
@@ -41,7 +41,7 @@ __device__ __forceinline__ void store_row_scale(const Params &p, uint32_t e, uin
         reinterpret_cast<float *>(sc)[row] = gs.s;
 }
 
-template <typename In, Kind KIND, bool FUSED, int SLOTS>
+template <typename In, Kind KIND, bool FUSED, int SLOTS, bool VARLEN>
 __global__ void __launch_bounds__(kRowThreads)
     row_quant_kernel(const __grid_constant__ Params p) {
     static_assert(!is_e2m1(KIND), "per-token E2M1 is not offered");
@@ -52,7 +52,7 @@ __global__ void __launch_bounds__(kRowThreads)
     const uint32_t lane = threadIdx.x & 31u;
     const uint32_t warp = threadIdx.x >> 5;
     // p.segs is 1 for this kernel: the table counts rows
-    const ExpertTable t = make_table(p, smem_prefix, lane);
+    const ExpertTable t = make_table<VARLEN>(p, smem_prefix, lane);
 
     const uint32_t wpr = p.items;               // warps per row: 1, 2, 4 or 8
     const uint32_t rows_per_iter = (kRowThreads / 32) / wpr;
@@ -67,8 +67,8 @@ __global__ void __launch_bounds__(kRowThreads)
          base += gridDim.x * rows_per_iter, parity ^= 1u) {
         const uint32_t r = base + sub;          // warp-uniform
         const bool live = r < t.total;
-        Span sp = locate(t, p.experts, live ? r : 0u);
-        const uint32_t row = (live ? r : 0u) - sp.start;
+        Span sp = locate<VARLEN>(t, p.experts, live ? r : 0u);
+        const uint32_t row = sp.base + ((live ? r : 0u) - sp.start);   // varlen: packed row
         const uint8_t *src = p.in + sp.e * p.in_expert_bytes +
                              static_cast<uint64_t>(row) * p.in_row_bytes;
 

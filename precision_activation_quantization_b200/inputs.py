@@ -93,10 +93,24 @@ class Workload:
     masked_m: np.ndarray | None = None   # int32 [E] or None (flat)
     expected_m: int = 0
     global_scale: float | None = None    # NVFP4 (scale_fmt "e4m3") only
+    # grouped-contiguous (varlen) calls: E == 1 plane of M packed rows holding
+    # len(seg_indptr) - 1 segments; seg_lens are token counts (or None)
+    seg_indptr: np.ndarray | None = None
+    seg_lens: np.ndarray | None = None
+
+    @property
+    def segments(self) -> int:
+        return 0 if self.seg_indptr is None else len(self.seg_indptr) - 1
 
     @property
     def rows(self) -> int:
-        """Rows actually quantized (tokens)."""
+        """Rows actually quantized (tokens).  For varlen calls this counts
+        the tokens of well-formed segments (increasing offsets within the M
+        rows, counts within each segment), the only kind generated here."""
+        if self.seg_indptr is not None:
+            if self.seg_lens is None:
+                return int(self.seg_indptr[-1] - self.seg_indptr[0])
+            return int(np.asarray(self.seg_lens, np.int64).sum())
         if self.masked_m is None:
             return self.E * self.M
         return int(np.clip(self.masked_m, 0, self.M).sum())
@@ -115,6 +129,9 @@ class Workload:
         else:
             scale_row = ng * (4 if self.scale_fmt == "fp32" else 1)
         extra = 0 if self.masked_m is None else 4 * self.E
+        if self.seg_indptr is not None:
+            extra += 4 * len(self.seg_indptr) + (0 if self.seg_lens is None
+                                                 else 4 * len(self.seg_lens))
         if self.global_scale is not None:
             extra += 4                   # the fp32 global scale
         return self.rows * (in_row + out_row + scale_row) + extra
@@ -214,3 +231,22 @@ def sweep(M: int, K: int = 4096, in_dtype: str = "bf16", group: int = 128,
     x = to_bits(laplace((M, K), seed), in_dtype).reshape(1, M, K)
     return Workload(f"sweep_{in_dtype}_{out_dtype}_g{group}_{M}x{K}", x, M=M, K=K,
                     group=group, in_dtype=in_dtype, out_dtype=out_dtype)
+
+
+def varlen(E: int = 32, M_max: int = 2048, K: int = 2048, seed: int = 4, count_seed: int = 5,
+           align: int = 128) -> Workload:
+    """Grouped-contiguous (varlen) dispatch with the fused prologue: the masked
+    workload's experts and token counts (masked_m[e] ~ U{0..M_max}, seed
+    ``count_seed``), packed into one buffer of [gate | up] rows whose segment e
+    holds its tokens followed by padding up to a multiple of ``align`` rows (the
+    M-block padding of a grouped-contiguous GEMM).  Tokens ~ N(0,1) ([seed]);
+    padding rows hold N(0,1) draws too (a consumer never reads them).
+    expected_m = the mean count rounded up."""
+    lens = np.random.default_rng(count_seed).integers(0, M_max + 1, size=E).astype(np.int32)
+    caps = -(-lens // align) * align
+    indptr = np.concatenate([[0], np.cumsum(caps)]).astype(np.int32)
+    M = int(indptr[-1])
+    x = bf16_bits(normal((1, M, 2 * K), seed))
+    return Workload(f"varlen_{E}x{M_max}x2x{K}", x, M=M, K=K, scale_fmt="ue8m0",
+                    layout="col", fused=True, expected_m=max(1, int(np.ceil(lens.mean()))),
+                    seg_indptr=indptr, seg_lens=lens)

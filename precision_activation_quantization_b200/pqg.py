@@ -37,8 +37,9 @@ SCALE_FMTS = {"fp32": PQG_SCALE_FP32, "ue8m0": PQG_SCALE_UE8M0, "e4m3": PQG_SCAL
 LAYOUTS = {"row": PQG_ROW_MAJOR, "col": PQG_COL_MAJOR_TMA, "packed": PQG_UE8M0_PACKED,
            "tile128x4": PQG_UE8M0_TILED_128x4}
 
-EXPORTS = ("pqg_quant", "pqg_quant_nvfp4", "pqg_scales_bytes", "pqg_status_string",
-           "pqg_last_cuda_error", "pqg_set_pdl", "pqg_launch_count", "pqg_version")
+EXPORTS = ("pqg_quant", "pqg_quant_nvfp4", "pqg_quant_varlen", "pqg_scales_bytes",
+           "pqg_status_string", "pqg_last_cuda_error", "pqg_set_pdl", "pqg_launch_count",
+           "pqg_version")
 
 
 class PqgError(RuntimeError):
@@ -59,6 +60,9 @@ def _load() -> ctypes.CDLL:
                               i64, vp]
     lib.pqg_quant_nvfp4.restype = i32
     lib.pqg_quant_nvfp4.argtypes = [vp, vp, vp, vp, i64, i64, i64, i32, i32, i32, vp, i64, vp]
+    lib.pqg_quant_varlen.restype = i32
+    lib.pqg_quant_varlen.argtypes = [vp, vp, vp, vp, i64, i64, i64, i32, i32, i32, i32, i32,
+                                     i32, vp, vp, i64, vp]
     lib.pqg_scales_bytes.restype = i64
     lib.pqg_scales_bytes.argtypes = [i64, i64, i64, i32, i32, i32]
     lib.pqg_status_string.restype = ctypes.c_char_p
@@ -96,6 +100,17 @@ def pqg_quant_nvfp4(in_ptr: int, out_ptr: int, scales_ptr: int, global_scale_ptr
     return _lib.pqg_quant_nvfp4(in_ptr, out_ptr, scales_ptr, global_scale_ptr, M, num_experts,
                                 K, in_dtype, scale_layout, fuse_silu_mul, masked_m_ptr,
                                 expected_m, stream)
+
+
+def pqg_quant_varlen(in_ptr: int, out_ptr: int, scales_ptr: int, global_scale_ptr: int | None,
+                     M: int, num_experts: int, K: int, group: int, in_dtype: int,
+                     out_dtype: int, scale_fmt: int, scale_layout: int, fuse_silu_mul: int,
+                     seg_indptr_ptr: int | None, seg_lens_ptr: int | None, expected_m: int,
+                     stream: int | None) -> int:
+    return _lib.pqg_quant_varlen(in_ptr, out_ptr, scales_ptr, global_scale_ptr, M, num_experts,
+                                 K, group, in_dtype, out_dtype, scale_fmt, scale_layout,
+                                 fuse_silu_mul, seg_indptr_ptr, seg_lens_ptr, expected_m,
+                                 stream)
 
 
 def pqg_scales_bytes(num_experts: int, M: int, K: int, group: int, scale_fmt: int,
@@ -280,4 +295,71 @@ def _launch(x, out, scales, M, E, K, group, in_dtype, out_dtype, scale_fmt, layo
                    getattr(stream, "cuda_stream", stream))
     if st != PQG_OK:
         raise PqgError(st)
+    return out, scales
+
+
+def quant_varlen(x, seg_indptr, seg_lens=None, out=None, scales=None, *, group: int = 128,
+                 out_dtype: str = "e4m3", scale_fmt: str = "fp32", layout: str = "row",
+                 fuse_silu_mul: bool = False, expected_m: int = 0, global_scale=None,
+                 stream=None):
+    """Grouped-contiguous (varlen) quantization of packed token rows; returns
+    (out, scales).
+
+    ``x`` is a contiguous bf16/fp16 CUDA tensor [M, K] ([M, 2K] when
+    ``fuse_silu_mul``) holding the segments of all experts.  ``seg_indptr`` is
+    an int32 CUDA tensor of E + 1 row offsets and ``seg_lens`` one of E token
+    counts (or None: every row of a segment is a token).  Token rows are
+    quantized into the same rows of ``out`` and of one scale plane of M rows;
+    padding rows are left as they are (``torch.empty`` when allocated here).
+    NVFP4 is ``out_dtype="e2m1", scale_fmt="e4m3", group=16`` with
+    ``global_scale``.  The call runs with ``x``'s device current.
+    """
+    import torch
+    if x.dtype not in (torch.bfloat16, torch.float16):
+        raise TypeError(f"unsupported input dtype {x.dtype}")
+    if not x.is_cuda or not x.is_contiguous() or x.dim() != 2:
+        raise ValueError("x must be a contiguous 2-D CUDA tensor of packed rows")
+    M, width = x.shape
+    K = width // 2 if fuse_silu_mul else width
+    E = seg_indptr.numel() - 1
+    for name, t, n in (("seg_indptr", seg_indptr, E + 1), ("seg_lens", seg_lens, E)):
+        if t is None:
+            continue
+        if (t.dtype != torch.int32 or t.device != x.device or t.numel() != n
+                or not t.is_contiguous()):
+            raise ValueError(f"{name} must be a contiguous int32 tensor of {n} entries on "
+                             f"x's device")
+    if E < 1:
+        raise ValueError("seg_indptr needs at least two entries")
+    if out is None or scales is None:
+        o, sc = allocate_outputs(M, K, group, out_dtype=out_dtype, scale_fmt=scale_fmt,
+                                 layout=layout, device=x.device)
+        out = o[0] if out is None else out
+        scales = sc[0] if scales is None else scales
+    out_bytes = M * (K // 2 if out_dtype == "e2m1" else K)
+    if out.numel() * out.element_size() != out_bytes or not out.is_contiguous():
+        raise ValueError(f"out must be a contiguous buffer of {out_bytes} bytes")
+    nbytes = pqg_scales_bytes(1, M, K, group, SCALE_FMTS[scale_fmt], LAYOUTS[layout])
+    if (nbytes >= 0 and scales.numel() * scales.element_size() != nbytes) \
+            or not scales.is_contiguous():
+        raise ValueError(f"scales must be a contiguous buffer of {nbytes} bytes")
+    if not (out.device == scales.device == x.device):
+        raise ValueError("x, out and scales must be on the same CUDA device")
+    gptr = None
+    if scale_fmt == "e4m3":
+        if (global_scale is None or global_scale.dtype != torch.float32
+                or global_scale.numel() != 1 or global_scale.device != x.device):
+            raise ValueError("NVFP4 needs global_scale: a one-element fp32 tensor on x's device")
+        gptr = global_scale.data_ptr()
+    if stream is None:
+        stream = torch.cuda.current_stream(x.device)
+    in_dtype = PQG_BF16 if x.dtype == torch.bfloat16 else PQG_FP16
+    with torch.cuda.device(x.device):
+        st = pqg_quant_varlen(x.data_ptr(), out.data_ptr(), scales.data_ptr(), gptr, M, E, K,
+                              group, in_dtype, OUT_DTYPES[out_dtype], SCALE_FMTS[scale_fmt],
+                              LAYOUTS[layout], int(bool(fuse_silu_mul)), seg_indptr.data_ptr(),
+                              None if seg_lens is None else seg_lens.data_ptr(),
+                              int(expected_m), getattr(stream, "cuda_stream", stream))
+    if st != PQG_OK:
+        raise PqgError(st, "pqg_quant_varlen")
     return out, scales

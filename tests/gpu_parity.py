@@ -38,7 +38,18 @@ def run_gpu(w, *, expected_m=None, stream=None, x_dev=None):
     mm = None if w.masked_m is None else torch.from_numpy(np.asarray(w.masked_m, np.int32)).cuda()
     s = stream if stream is not None else torch.cuda.current_stream()
     em = w.expected_m if expected_m is None else expected_m
-    if w.scale_fmt == "e4m3":
+    if w.seg_indptr is not None:
+        ip = torch.from_numpy(np.asarray(w.seg_indptr, np.int32)).cuda()
+        ln = None if w.seg_lens is None else torch.from_numpy(np.asarray(w.seg_lens, np.int32)).cuda()
+        gsc = (torch.tensor([w.global_scale], dtype=torch.float32, device="cuda")
+               if w.scale_fmt == "e4m3" else None)
+        st = pqg.pqg_quant_varlen(x.data_ptr(), out.data_ptr(), sc.data_ptr(),
+                                  None if gsc is None else gsc.data_ptr(), w.M, w.segments,
+                                  w.K, w.group, pqg.IN_DTYPES[w.in_dtype],
+                                  pqg.OUT_DTYPES[w.out_dtype], pqg.SCALE_FMTS[w.scale_fmt],
+                                  pqg.LAYOUTS[w.layout], int(w.fused), ip.data_ptr(),
+                                  None if ln is None else ln.data_ptr(), em, s.cuda_stream)
+    elif w.scale_fmt == "e4m3":
         gsc = torch.tensor([w.global_scale], dtype=torch.float32, device="cuda")
         st = pqg.pqg_quant_nvfp4(x.data_ptr(), out.data_ptr(), sc.data_ptr(), gsc.data_ptr(),
                                  w.M, w.E, w.K, pqg.IN_DTYPES[w.in_dtype],
@@ -59,6 +70,13 @@ def run_gpu(w, *, expected_m=None, stream=None, x_dev=None):
 
 def run_oracle(w):
     """The oracle's (codes uint8 [E*M*K], scale bytes), sentinel-filled like run_gpu."""
+    if w.seg_indptr is not None:
+        q, s = oracle.quant_varlen(w.x, M=w.M, K=w.K, group=w.group, seg_indptr=w.seg_indptr,
+                                   seg_lens=w.seg_lens, in_dtype=w.in_dtype,
+                                   out_dtype=w.out_dtype, scale_fmt=w.scale_fmt,
+                                   layout=w.layout, fused=w.fused, fill=SENTINEL,
+                                   global_scale=w.global_scale)
+        return q.reshape(-1), s.view(np.uint8).reshape(-1)
     q, s = oracle.quant(w.x, E=w.E, M=w.M, K=w.K, group=w.group, in_dtype=w.in_dtype,
                         out_dtype=w.out_dtype, scale_fmt=w.scale_fmt, layout=w.layout,
                         fused=w.fused, masked_m=w.masked_m, fill=SENTINEL,
@@ -165,8 +183,11 @@ def check_fused(w, *, max_flip_frac=CONTRACT_FLIP_FRAC, rel_tol=7e-2, **kw):
     gq, gs = run_gpu(w, **kw)
     rq, rs = run_oracle(w)
     E, M, K, G = w.E, w.M, w.K, w.group
-    rows = np.full(E, M) if w.masked_m is None else np.clip(w.masked_m, 0, M)
-    live = np.arange(M)[None, :] < rows[:, None]                       # [E, M]
+    if w.seg_indptr is not None:                                       # varlen: one plane
+        live = oracle.varlen_rows(w.seg_indptr, w.seg_lens, M)[None, :]
+    else:
+        rows = np.full(E, M) if w.masked_m is None else np.clip(w.masked_m, 0, M)
+        live = np.arange(M)[None, :] < rows[:, None]                   # [E, M]
 
     # untouched rows and padding must be byte-identical (sentinels)
     kb = K // 2 if w.out_dtype == "e2m1" else K
@@ -193,7 +214,7 @@ def check_fused(w, *, max_flip_frac=CONTRACT_FLIP_FRAC, rel_tol=7e-2, **kw):
             m_of, e_of = elem % mpad, elem // (ng * mpad)
         else:
             m_of, e_of = (elem // ng) % M, elem // (M * ng)
-    inside = m_of < rows[e_of]
+    inside = (m_of < M) & live[e_of, np.minimum(m_of, max(M - 1, 0))]
     assert_same(gs[~inside], rs[~inside], f"{w.name} untouched scale bytes")
     if w.layout == "packed":
         j = (idx // 4 // mpad) % ((ng + 3) // 4)

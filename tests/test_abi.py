@@ -235,6 +235,51 @@ def test_nvfp4_rejects_before_launch(kw, status):
     assert pqg.pqg_launch_count() == before
 
 
+def call_var(**kw):
+    a = dict(in_ptr=FAKE, out_ptr=FAKE + (1 << 32), scales_ptr=FAKE + (2 << 32),
+             global_scale_ptr=None, M=64, num_experts=4, K=256, group=128,
+             in_dtype=pqg.PQG_BF16, out_dtype=pqg.PQG_E4M3, scale_fmt=pqg.PQG_SCALE_UE8M0,
+             scale_layout=pqg.PQG_COL_MAJOR_TMA, fuse_silu_mul=1,
+             seg_indptr_ptr=FAKE + (3 << 32), seg_lens_ptr=FAKE + (4 << 32), expected_m=8,
+             stream=None)
+    a.update(kw)
+    return pqg.pqg_quant_varlen(**a)
+
+
+@host_only
+@pytest.mark.parametrize("kw,status", [
+    (dict(seg_indptr_ptr=0), pqg.PQG_ERR_INVALID_ARG),
+    (dict(seg_indptr_ptr=0, M=0), pqg.PQG_ERR_INVALID_ARG),         # needed even with no rows
+    (dict(seg_indptr_ptr=FAKE + (3 << 32) + 2), pqg.PQG_ERR_ALIGNMENT),
+    (dict(seg_lens_ptr=FAKE + (4 << 32) + 1), pqg.PQG_ERR_ALIGNMENT),
+    (dict(num_experts=0), pqg.PQG_ERR_INVALID_ARG),
+    (dict(num_experts=4097), pqg.PQG_ERR_INVALID_ARG),
+    (dict(M=-1), pqg.PQG_ERR_INVALID_ARG),
+    (dict(M=1 << 31), pqg.PQG_ERR_INVALID_ARG),
+    (dict(K=200), pqg.PQG_ERR_INVALID_ARG),
+    (dict(group=16), pqg.PQG_ERR_UNSUPPORTED),
+    (dict(out_dtype=pqg.PQG_INT8), pqg.PQG_ERR_UNSUPPORTED),       # INT8 with UE8M0
+    (dict(global_scale_ptr=FAKE + (5 << 32)), pqg.PQG_ERR_INVALID_ARG),   # g without NVFP4
+    (dict(out_dtype=pqg.PQG_E2M1, scale_fmt=pqg.PQG_SCALE_E4M3, group=16),
+     pqg.PQG_ERR_INVALID_ARG),                                      # NVFP4 without g
+    (dict(in_ptr=FAKE + 16), pqg.PQG_ERR_ALIGNMENT),
+    (dict(out_ptr=FAKE + 1024), pqg.PQG_ERR_INVALID_ARG),           # overlaps the input
+    (dict(seg_indptr_ptr=FAKE + (1 << 32) + 64), pqg.PQG_ERR_INVALID_ARG),   # inside out
+    (dict(seg_lens_ptr=FAKE + (2 << 32) + 4), pqg.PQG_ERR_INVALID_ARG),      # inside scales
+])
+def test_varlen_rejects_before_launch(kw, status):
+    before = pqg.pqg_launch_count()
+    assert call_var(**kw) == status
+    assert pqg.pqg_launch_count() == before
+
+
+@host_only
+def test_varlen_zero_rows_is_ok_and_launches_nothing():
+    before = pqg.pqg_launch_count()
+    assert call_var(M=0, in_ptr=0, out_ptr=0, scales_ptr=0) == pqg.PQG_OK
+    assert pqg.pqg_launch_count() == before
+
+
 @host_only
 def test_quant_refers_e4m3_block_scales_to_the_nvfp4_entry():
     assert call(out_dtype=pqg.PQG_E2M1, scale_fmt=pqg.PQG_SCALE_E4M3,

@@ -194,3 +194,38 @@ def test_fused_check_catches_codes_in_an_nvfp4_zero_block(monkeypatch):
     _device_returns(monkeypatch, code)
     with pytest.raises(AssertionError, match="nonzero codes in zero blocks"):
         check_fused(w, max_flip_frac=1e-3)
+
+
+def _varlen_fused(layout="col", fmt="ue8m0"):
+    from test_parity_gpu import make_var
+    return make_var([0, 16, 16, 48], [9, 0, 30], 256, 128, ("e4m3", fmt, layout), fused=True,
+                    seed=7, M=52)
+
+
+@pytest.mark.parametrize("layout,fmt", [("col", "ue8m0"), ("packed", "ue8m0"), ("row", "fp32"),
+                                        ("tile128x4", "ue8m0")])
+def test_varlen_oracle_bytes_pass_and_padding_writes_fail(monkeypatch, layout, fmt):
+    """Varlen calls: the oracle's bytes pass both checks; a code written into a
+    padding row (row 12 of segment 0), or a scale cell of a row in no segment,
+    fails."""
+    w = _varlen_fused(layout, fmt)
+    _device_returns(monkeypatch)
+    assert check_fused(w)["flip_frac"] == 0.0
+    check_exact(w.with_(fused=False, x=w.x[..., :256].copy()))
+    _device_returns(monkeypatch, lambda w, q, s: q.__setitem__(12 * 256 + 3, 0x11))
+    with pytest.raises(AssertionError, match="masked-off codes"):
+        check_fused(w)
+    ng = 2
+
+    def scale_cell(w, q, s):
+        if layout == "row":
+            s[(50 * ng) * 4] ^= 1                  # fp32 scale of row 50 (in no segment)
+        elif layout == "col":
+            s[0 * 52 + 50] ^= 1                    # group 0 of row 50
+        elif layout == "packed":
+            s[50 * 4] ^= 1                         # word 0 of row 50
+        else:
+            s[(50 % 32) * 16 + (50 // 32) * 4] ^= 1
+    _device_returns(monkeypatch, scale_cell)
+    with pytest.raises(AssertionError, match="untouched scale bytes"):
+        check_fused(w)

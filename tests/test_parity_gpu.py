@@ -399,33 +399,131 @@ def test_per_token_full_size():
 # grouped-contiguous (varlen) tokens: a flat call over the packed rows
 # --------------------------------------------------------------------------
 
-@pytest.mark.parametrize("kind", [("e4m3", "ue8m0", "row"), ("e4m3", "fp32", "row")],
-                         ids=lambda k: "_".join(k))
-def test_varlen_contiguous_equals_masked(kind):
-    """The tokens of each expert packed back to back (blocks padded to 128 rows,
-    as a grouped-contiguous GEMM takes them) quantize, with one flat fused call,
-    to the same bytes as masked dispatch over [E, M_max, 2K]."""
+# --------------------------------------------------------------------------
+# grouped-contiguous (varlen): token segments packed in one buffer
+# --------------------------------------------------------------------------
+
+def make_var(indptr, lens, K, G, kind, in_dtype="bf16", fused=False, seed=0, M=None,
+             expected_m=0, global_scale=None):
+    """A varlen workload over M packed rows (default: the last offset) with the
+    given segments; every row, padding included, holds adversarial values."""
+    indptr = np.asarray(indptr, np.int32)
+    M = int(indptr[-1]) if M is None else M
+    w = make(M, K, G, kind, in_dtype, fused=fused, seed=seed, expected_m=expected_m)
+    return w.with_(name=f"varlen_{w.name}_E{len(indptr) - 1}", seg_indptr=indptr,
+                   seg_lens=None if lens is None else np.asarray(lens, np.int32),
+                   global_scale=global_scale)
+
+
+# (indptr, lens, M): padded segments, an empty one, a count past its segment,
+# no counts, a negative count, offsets out of range, rows in no segment
+VARLEN_SEGMENTS = [
+    ([0, 128, 128, 384, 512], [100, 0, 300, 37], None),
+    ([0, 5, 9, 16, 23], None, None),
+    ([0, 40, 41, 80], [-3, 1, 39], 84),
+    ([-8, 16, 12, 70], [20, 5, 50], 64),
+]
+
+
+@pytest.mark.parametrize("kind", KINDS, ids=lambda k: "_".join(k))
+@pytest.mark.parametrize("seg", range(len(VARLEN_SEGMENTS)))
+def test_varlen_variants(kind, seg):
+    """Token rows match the oracle bit for bit (plain) or within the fused
+    contract; padding rows and rows in no segment keep the sentinel."""
+    indptr, lens, M = VARLEN_SEGMENTS[seg]
+    for fused in (False, True):
+        for G, K in ((128, 640), (32, 1536)):
+            w = make_var(indptr, lens, K, G, kind, fused=fused, seed=seg * 7 + G + fused, M=M,
+                         expected_m=16)
+            if fused:
+                check_fused(w, max_flip_frac=1e-3)
+            else:
+                check_exact(w)
+
+
+@pytest.mark.parametrize("E", [1, 33, 300, 4096])
+def test_varlen_expert_table_modes(E):
+    """One segment, the warp-register table (<= 32), and the shared-memory table
+    (more than 32 segments, up to 4096) with their first rows."""
+    rng = np.random.default_rng(E)
+    lens = rng.integers(0, 9, size=E).astype(np.int32)
+    caps = lens + rng.integers(0, 3, size=E).astype(np.int32)
+    indptr = np.concatenate([[0], np.cumsum(caps)]).astype(np.int32)
+    check_exact(make_var(indptr, lens, 256, 64, ("e4m3", "ue8m0", "packed"), seed=E))
+    check_exact(make_var(indptr, lens, 384, 128, ("int8", "fp32", "col"), in_dtype="fp16",
+                         seed=E + 1))
+    check_fused(make_var(indptr, lens, 512, 128, ("e4m3", "fp32", "row"), fused=True,
+                         seed=E + 2), max_flip_frac=1e-3)
+
+
+@pytest.mark.parametrize("K", [512, 7168])
+def test_varlen_per_token(K):
+    indptr, lens, M = VARLEN_SEGMENTS[0]
+    check_exact(make_var(indptr, lens, K, K, ("e4m3", "fp32", "row"), seed=K))
+    check_exact(make_var(indptr, lens, K, K, ("e4m3", "ue8m0", "packed"), in_dtype="fp16",
+                         seed=K + 1))
+    check_fused(make_var(indptr, lens, K, K, ("e4m3", "fp32", "col"), fused=True, seed=K + 2),
+                max_flip_frac=1e-3)
+    check_exact(make_var([0, 60, 200], [60, 100], K, K, ("int8", "fp32", "row"), seed=K + 3))
+
+
+@pytest.mark.parametrize("layout", ["row", "col", "tile128x4"])
+def test_varlen_fp4(layout):
+    """MXFP4 (G = 32, UE8M0) and NVFP4 (blocks of 16 under a global scale)."""
+    indptr, lens, M = VARLEN_SEGMENTS[0]
+    check_exact(make_var(indptr, lens, 640, 32, ("e2m1", "ue8m0", layout), seed=81))
+    check_fused(make_var(indptr, lens, 640, 32, ("e2m1", "ue8m0", layout), fused=True,
+                         seed=82), max_flip_frac=1e-3)
+    nv = ("e2m1", "e4m3", layout)
+    check_exact(make_var(indptr, lens, 640, 16, nv, seed=83, global_scale=2.625))
+    check_fused(make_var(indptr, lens, 640, 16, nv, fused=True, seed=84, global_scale=2.625),
+                max_flip_frac=1e-3)
+
+
+def test_varlen_expected_m_does_not_change_results():
+    indptr, lens, M = VARLEN_SEGMENTS[0]
+    w = make_var(indptr, lens, 1024, 128, ("e4m3", "ue8m0", "packed"), seed=90)
+    ref = run_gpu(w, expected_m=0)
+    for em in (1, 7, 100, 10 ** 6, -5):
+        got = run_gpu(w, expected_m=em)
+        assert_same(got[0], ref[0], f"codes, expected_m={em}")
+        assert_same(got[1], ref[1], f"scales, expected_m={em}")
+
+
+def test_varlen_full_size():
+    """The varlen workload: the masked workload's 32 experts and token counts
+    (30 218 tokens) packed in segments padded to 128 rows, fused SiLU-and-mul,
+    E4M3 codes, UE8M0 column-major scales over the 32 256 packed rows."""
+    check_fused(inputs.varlen())
+
+
+def test_varlen_equals_masked_over_the_same_tokens():
+    """The same tokens through masked dispatch ([E, M_max, 2K]) and varlen
+    dispatch (segments padded to 128 rows) give the same codes and row-major
+    scales on the GPU, and each matches the oracle."""
     E, M_max, K = 4, 256, 1024
     counts = np.array([100, 0, 256, 37], np.int32)
+    kind = ("e4m3", "ue8m0", "row")
     w = make(M_max, K, 128, kind, fused=True, E=E, seed=41, masked_m=counts, expected_m=100)
-    mq, ms = run_gpu(w)
-    mq = mq.reshape(E, M_max, K)
-    ms = ms.view(np.float32 if kind[1] == "fp32" else np.uint8).reshape(E, M_max, K // 128)
-    blocks = [(-(-int(c) // 128)) * 128 for c in counts]
-    packed = np.zeros((1, sum(blocks), 2 * K), np.uint16)
-    off = np.concatenate([[0], np.cumsum(blocks)])
+    caps = -(-counts // 128) * 128
+    indptr = np.concatenate([[0], np.cumsum(caps)]).astype(np.int32)
+    packed = np.zeros((1, int(indptr[-1]), 2 * K), np.uint16)
     for e in range(E):
-        packed[0, off[e]:off[e] + counts[e]] = w.x[e, :counts[e]]
-    flat = inputs.Workload("varlen", packed, M=sum(blocks), K=K, group=128, out_dtype=kind[0],
-                           scale_fmt=kind[1], layout="row", fused=True)
-    fq, fs = run_gpu(flat)
-    fq = fq.reshape(-1, K)
-    fs = fs.view(np.float32 if kind[1] == "fp32" else np.uint8).reshape(-1, K // 128)
+        packed[0, indptr[e]:indptr[e] + counts[e]] = w.x[e, :counts[e]]
+    v = inputs.Workload("varlen_packed", packed, M=int(indptr[-1]), K=K, group=128,
+                        out_dtype="e4m3", scale_fmt="ue8m0", layout="row", fused=True,
+                        seg_indptr=indptr, seg_lens=counts)
+    check_fused(w, max_flip_frac=1e-3)
+    check_fused(v, max_flip_frac=1e-3)
+    mq, ms = run_gpu(w)
+    vq, vs = run_gpu(v)
+    mq, ms = mq.reshape(E, M_max, K), ms.reshape(E, M_max, K // 128)
+    vq, vs = vq.reshape(-1, K), vs.reshape(-1, K // 128)
     for e in range(E):
         n = int(counts[e])
-        assert_same(fq[off[e]:off[e] + n].reshape(-1), mq[e, :n].reshape(-1), f"codes e={e}")
-        assert_same(fs[off[e]:off[e] + n].view(np.uint8).reshape(-1),
-                    ms[e, :n].view(np.uint8).reshape(-1), f"scales e={e}")
+        assert_same(vq[indptr[e]:indptr[e] + n], mq[e, :n], f"codes e={e}")
+        assert_same(vs[indptr[e]:indptr[e] + n], ms[e, :n], f"scales e={e}")
+        assert (vq[indptr[e] + n:indptr[e + 1]] == SENTINEL).all()
 
 
 # --------------------------------------------------------------------------

@@ -11,6 +11,7 @@
 #include <type_traits>
 
 #include "pqg_kernel.cuh"
+#include "pqg_pipe_kernel.cuh"
 #include "pqg_row_kernel.cuh"
 
 namespace pqg {
@@ -29,6 +30,34 @@ struct LaunchArgs {
 };
 
 int sm_count(int device);  // cached cudaDevAttrMultiProcessorCount
+
+// Resident CTAs per SM of one kernel variant, cached per device: the
+// occupancy query (and the shared-memory attribute it needs) applies to the
+// current device, so a process driving several devices queries each once.
+constexpr int kOccDevices = 64;
+struct OccupancyCache {
+    std::atomic<int> n[kOccDevices][2];   // [device][0: no table, 1: largest table]; 0 = unknown
+};
+
+template <typename Kernel>
+inline int blocks_per_sm(OccupancyCache &cache, Kernel kernel, int device, int threads,
+                         uint32_t max_smem, uint32_t smem) {
+    const int which = smem == 0 ? 0 : 1;
+    const bool cached = device >= 0 && device < kOccDevices;
+    if (cached) {
+        const int n = cache.n[device][which].load(std::memory_order_relaxed);
+        if (n > 0) return n;
+    }
+    int n = 0;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(max_smem)) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, threads,
+                                                      which ? max_smem : 0u) != cudaSuccess ||
+        n < 1)
+        n = 1;
+    if (cached) cache.n[device][which].store(n, std::memory_order_relaxed);
+    return n;
+}
 
 // Strips per register chunk (ITEMS) and warps per CTA, tunable at build time.
 // Each lane issues ITEMS 32-byte loads (twice that fused) per chunk.
@@ -113,25 +142,14 @@ cudaError_t launch_variant(const LaunchArgs &a) {
     constexpr bool kVar = DISP == kVarlen;
     auto kernel = quant_kernel<In, G, KIND, FUSED, kItems, kWarps, DISP>;
 
-    // Resident CTAs per SM, queried once per variant without and with the
-    // largest shared-memory expert table (more than 32 experts).
-    static const int2 occupancy = [&] {
-        int n0 = 0, n1 = 0;
-        if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(smem_bytes(kMaxExperts, kVar))) != cudaSuccess ||
-            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n0, kernel, kThreads, 0) !=
-                cudaSuccess ||
-            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n1, kernel, kThreads,
-                                                          smem_bytes(kMaxExperts, kVar)) !=
-                cudaSuccess)
-            n0 = n1 = 1;
-        return make_int2(n0 < 1 ? 1 : n0, n1 < 1 ? 1 : n1);
-    }();
-    const int blocks_per_sm = smem_bytes(a.p.experts, kVar) == 0 ? occupancy.x : occupancy.y;
-
     int device = 0;
     cudaError_t err = cudaGetDevice(&device);
     if (err != cudaSuccess) return err;
+    // Resident CTAs per SM on this device, without or with the largest
+    // shared-memory expert table (more than 32 experts).
+    static OccupancyCache cache;
+    const int bps = blocks_per_sm(cache, kernel, device, kThreads, smem_bytes(kMaxExperts, kVar),
+                                  smem_bytes(a.p.experts, kVar));
 
     // Strips per warp: ITEMS, or 1 when the expected work would not fill one
     // wave (latency-bound calls spread over more SMs).  Grid: one CTA per
@@ -139,7 +157,7 @@ cudaError_t launch_variant(const LaunchArgs &a) {
     // waves of blocks) runs one resident wave that loops over the blocks (no
     // ragged last wave), and a long one at most PQG_WAVES waves.  Blocks are
     // taken round-robin, so any real total is covered.
-    const uint64_t wave = static_cast<uint64_t>(sm_count(device)) * blocks_per_sm;
+    const uint64_t wave = static_cast<uint64_t>(sm_count(device)) * bps;
     Params p = a.p;
     p.items = kItems;
     if (a.expected_strips < wave * kWarps * kItems) p.items = 1;
@@ -163,6 +181,51 @@ cudaError_t launch_variant(const LaunchArgs &a) {
     return cudaLaunchKernelEx(&cfg, kernel, p);
 }
 
+// Flat fused calls through the shared-memory pipelined kernel
+// (pqg_pipe_kernel.cuh): warps per CTA, strips per warp in the pipeline, and
+// the grid in waves of resident CTAs.
+#ifndef PQG_FUSED_PIPE
+#define PQG_FUSED_PIPE 0
+#endif
+#ifndef PQG_PIPE_WARPS
+#define PQG_PIPE_WARPS 4
+#endif
+#ifndef PQG_PIPE_STAGES
+#define PQG_PIPE_STAGES 2
+#endif
+#ifndef PQG_PIPE_WAVES
+#define PQG_PIPE_WAVES 1
+#endif
+
+template <typename In, int G, Kind KIND>
+cudaError_t launch_pipe(const LaunchArgs &a) {
+    constexpr int kWarps = PQG_PIPE_WARPS, kStages = PQG_PIPE_STAGES;
+    constexpr uint32_t kSmem = pipe_smem_bytes(kWarps, kStages);
+    auto kernel = fused_pipe_kernel<In, G, KIND, kWarps, kStages>;
+    int device = 0;
+    cudaError_t err = cudaGetDevice(&device);
+    if (err != cudaSuccess) return err;
+    static OccupancyCache cache;
+    const int bps = blocks_per_sm(cache, kernel, device, kWarps * 32, kSmem, kSmem);
+    const uint64_t wave = static_cast<uint64_t>(sm_count(device)) * bps;
+    uint64_t ctas = (a.expected_strips + kWarps - 1) / kWarps;
+    if (ctas > wave * PQG_PIPE_WAVES) ctas = wave * PQG_PIPE_WAVES;
+    if (ctas < 1) ctas = 1;
+    Params p = a.p;
+    p.items = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(ctas), 1, 1);
+    cfg.blockDim = dim3(kWarps * 32, 1, 1);
+    cfg.dynamicSmemBytes = kSmem;
+    cfg.stream = a.stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = a.pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kernel, p);
+}
+
 template <typename In, int G, Kind KIND>
 cudaError_t launch_kind(const LaunchArgs &a) {
     if (a.disp == kVarlen)
@@ -171,6 +234,7 @@ cudaError_t launch_kind(const LaunchArgs &a) {
     const bool multi = a.p.experts > 1;
     if (a.fused) {
         if (multi) return launch_variant<In, G, KIND, true, kMasked>(a);
+        if constexpr (PQG_FUSED_PIPE != 0) return launch_pipe<In, G, KIND>(a);
         // A long flat fused call (4 or more waves of 1-strip work at 48 warps
         // per SM) runs a variant compiled for 2 strips per chunk: [4096, 2 x
         // 7168] 26.4 -> 24.6 us.  Short calls keep the 1-strip variant, whose
@@ -232,28 +296,20 @@ inline void row_shape(uint32_t K, uint32_t *wpr, int *slots) {
 template <typename In, Kind KIND, bool FUSED, int SLOTS, bool VARLEN>
 cudaError_t launch_row_variant(const LaunchArgs &a, uint32_t wpr) {
     auto kernel = row_quant_kernel<In, KIND, FUSED, SLOTS, VARLEN>;
-    static const int blocks_per_sm = [&] {
-        int n = 0;
-        if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(smem_bytes(kMaxExperts, VARLEN))) !=
-                cudaSuccess ||
-            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, kRowThreads,
-                                                          smem_bytes(kMaxExperts, VARLEN)) !=
-                cudaSuccess ||
-            n < 1)
-            n = 1;
-        return n;
-    }();
     int device = 0;
     cudaError_t err = cudaGetDevice(&device);
     if (err != cudaSuccess) return err;
+    // sized with the largest expert table, whatever this call's table
+    static OccupancyCache cache;
+    const int bps = blocks_per_sm(cache, kernel, device, kRowThreads,
+                                  smem_bytes(kMaxExperts, VARLEN), smem_bytes(kMaxExperts, VARLEN));
 
     Params p = a.p;
     p.segs = 1;        // the expert table counts rows
     p.items = wpr;     // warps per row
     const uint64_t rows_per_cta = (kRowThreads / 32) / wpr;
     uint64_t ctas = (a.expected_rows + rows_per_cta - 1) / rows_per_cta;
-    const uint64_t cap = static_cast<uint64_t>(sm_count(device)) * blocks_per_sm * PQG_ROW_WAVES;
+    const uint64_t cap = static_cast<uint64_t>(sm_count(device)) * bps * PQG_ROW_WAVES;
     if (ctas > cap) ctas = cap;
     if (ctas < 1) ctas = 1;
 

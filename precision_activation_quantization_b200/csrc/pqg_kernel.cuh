@@ -153,6 +153,12 @@ __device__ __forceinline__ void load32B(const void *p, uint32_t (&r)[8]) {
         : "l"(p));
 }
 
+// Bring `bytes` bytes (a multiple of 16, 16-byte aligned) into L2 with the
+// bulk-copy engine: one instruction, no registers, no completion to wait for.
+__device__ __forceinline__ void prefetch_l2(const void *p, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
 __device__ __forceinline__ void store8B(void *p, uint32_t a, uint32_t b) {
     asm volatile("st.global.v2.b32 [%0], {%1,%2};" ::"l"(p), "r"(a), "r"(b) : "memory");
 }
@@ -205,12 +211,21 @@ __device__ __forceinline__ void widen2<__half>(uint32_t w, float &lo, float &hi)
     hi = f.y;
 }
 
-// silu(g) * u for a pair, in fp32: sigmoid(g) = 1 / (1 + 2^(-g * log2 e)) with
-// the hardware ex2 and rcp approximations, on packed f32x2 arithmetic where it
-// exists.  The extremes stay right without a branch: for g << 0 the power is
-// +inf (or the reciprocal flushes to zero) and silu is a zero of g's sign; for
-// g >> 0 the power flushes to 0 and sigmoid is 1.  The product stays within a
-// few fp32 ulps of silu(g) * u.
+// silu(g) * u for a pair, in fp32: sigmoid(g) = 1 / (1 + 2^t), t = -g log2 e,
+// with the hardware ex2 and rcp approximations, on packed f32x2 arithmetic
+// where it exists.  g * u is one exact mixed-precision FMA of the two 16-bit
+// inputs (8- or 11-bit significands: the product fits fp32), so the element is
+// (g u) / (1 + 2^t) with the approximations' errors and one rounding.  The
+// extremes stay right without a branch: for g << 0 the power is +inf (or the
+// reciprocal flushes to zero) and the result is a zero with g u's sign; for
+// g >> 0 the power flushes to 0 and the result is g u.  The product stays
+// within a few fp32 ulps of silu(g) * u.
+//
+// Both approximations run on the SFU (MUFU) pipe, about 60 % busy at the
+// hidden-size fused call.  Moving the reciprocal to the FMA pipe (an integer
+// seed and three Newton-Raphson steps on f32x2 FMAs) was measured slower: the
+// eight extra instructions per pair cost more than the freed SFU slot
+// ([4096, 2 x 7168] 25.1 -> 26.3 us, masked 51.4 -> 55.6 us).
 __device__ __forceinline__ float ex2_approx(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -221,13 +236,35 @@ __device__ __forceinline__ float rcp_approx(float x) {
     asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
 }
-__device__ __forceinline__ float2 silu_mul2(float2 g, float2 u) {
+// a * b for the 16-bit halves of two packed words, exact in fp32 (adding -0
+// keeps every product, -0 included)
+template <typename In>
+__device__ __forceinline__ float2 mul_exact2(uint32_t a, uint32_t b) {
+    float lo, hi;
+    if constexpr (std::is_same<In, __nv_bfloat16>::value)
+        asm("{\n\t.reg .b16 al, ah, bl, bh;\n\t"
+            "mov.b32 {al, ah}, %2;\n\tmov.b32 {bl, bh}, %3;\n\t"
+            "fma.rn.f32.bf16 %0, al, bl, 0f80000000;\n\t"
+            "fma.rn.f32.bf16 %1, ah, bh, 0f80000000;\n\t}"
+            : "=f"(lo), "=f"(hi) : "r"(a), "r"(b));
+    else
+        asm("{\n\t.reg .b16 al, ah, bl, bh;\n\t"
+            "mov.b32 {al, ah}, %2;\n\tmov.b32 {bl, bh}, %3;\n\t"
+            "fma.rn.f32.f16 %0, al, bl, 0f80000000;\n\t"
+            "fma.rn.f32.f16 %1, ah, bh, 0f80000000;\n\t}"
+            : "=f"(lo), "=f"(hi) : "r"(a), "r"(b));
+    return make_float2(lo, hi);
+}
+// silu(gate) * up for the pair of elements held in packed words gw and uw
+template <typename In>
+__device__ __forceinline__ float2 silu_mul_pair(uint32_t gw, uint32_t uw) {
     constexpr float kNegLog2e = -1.4426950408889634f;
-    const float2 t = __fmul2_rn(g, make_float2(kNegLog2e, kNegLog2e));
+    float g0, g1;
+    widen2<In>(gw, g0, g1);
+    const float2 t = __fmul2_rn(make_float2(g0, g1), make_float2(kNegLog2e, kNegLog2e));
     const float2 d = __fadd2_rn(make_float2(ex2_approx(t.x), ex2_approx(t.y)),
                                 make_float2(1.0f, 1.0f));
-    const float2 sig = make_float2(rcp_approx(d.x), rcp_approx(d.y));
-    return __fmul2_rn(__fmul2_rn(g, sig), u);
+    return __fmul2_rn(mul_exact2<In>(gw, uw), make_float2(rcp_approx(d.x), rcp_approx(d.y)));
 }
 
 // Packed pair of E4M3 codes: `lo` in bits 0-7, `hi` in bits 8-15.  Round to
@@ -710,6 +747,56 @@ __device__ __forceinline__ void load_chunk(Chunk<ITEMS, FUSED> &ch, uint32_t s, 
     }
 }
 
+// Prefetch into L2 the strips [s, s + n) a warp takes next (one bulk prefetch
+// per strip and half, issued by lane 0), so that their loads, issued after this
+// chunk's arithmetic, find them there.  Used by looping grids.
+#ifndef PQG_PREFETCH_STRIP
+#define PQG_PREFETCH_STRIP 0
+#endif
+template <int ITEMS, bool FUSED, int DISP>
+__device__ __forceinline__ void prefetch_chunk(uint32_t s, uint32_t n, const ExpertTable &t,
+                                               const Params &p, uint32_t lane) {
+    constexpr bool kVar = DISP == kVarlen;
+    uint32_t e = 0, start = 0, end_e = t.total, base = 0;
+    if constexpr (DISP != kFlat) {
+        const Span sp = locate<kVar>(t, p.experts, s);
+        e = sp.e;
+        start = sp.start;
+        end_e = sp.start + sp.strips;
+        base = sp.base;
+    }
+    uint32_t row = (s - start) / p.segs;
+    uint32_t seg = (s - start) - row * p.segs;
+#pragma unroll
+    for (int k = 0; k < ITEMS; ++k) {
+        if (static_cast<uint32_t>(k) >= n) break;      // warp-uniform
+        if constexpr (DISP != kFlat) {
+            if (s + k >= end_e) {
+                const Span sp = locate<kVar>(t, p.experts, s + k);
+                e = sp.e;
+                start = sp.start;
+                end_e = sp.start + sp.strips;
+                base = sp.base;
+                row = 0;
+                seg = 0;
+            }
+        }
+        if (lane == 0) {
+            const uint32_t col0 = seg * kStripElems;
+            const uint32_t bytes = min(kStripBytes, (p.K - col0) * 2u);
+            const uint8_t *src = p.in + e * p.in_expert_bytes +
+                                 static_cast<uint64_t>(base + row) * p.in_row_bytes +
+                                 static_cast<uint64_t>(col0) * 2u;
+            prefetch_l2(src, bytes);
+            if constexpr (FUSED) prefetch_l2(src + static_cast<uint64_t>(p.K) * 2u, bytes);
+        }
+        if (++seg == p.segs) {
+            seg = 0;
+            ++row;
+        }
+    }
+}
+
 // bf16 UE8M0 through the mixed-precision FMA path (1) or by widening (0).
 #ifndef PQG_UE8M0_MIXED
 #define PQG_UE8M0_MIXED 1
@@ -761,13 +848,12 @@ __device__ __forceinline__ void quantize_strip(const uint32_t (&x)[8], const uin
         float v[16];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-            widen2<In>(x[i], v[2 * i], v[2 * i + 1]);
             if constexpr (FUSED) {
-                float u0, u1;
-                widen2<In>(u[i], u0, u1);
-                const float2 y = silu_mul2(make_float2(v[2 * i], v[2 * i + 1]), make_float2(u0, u1));
+                const float2 y = silu_mul_pair<In>(x[i], u[i]);
                 v[2 * i] = y.x;
                 v[2 * i + 1] = y.y;
+            } else {
+                widen2<In>(x[i], v[2 * i], v[2 * i + 1]);
             }
         }
         float amax = 0.0f;
@@ -782,10 +868,14 @@ __device__ __forceinline__ void quantize_strip(const uint32_t (&x)[8], const uin
     uint32_t packed_word = 0;
     if constexpr (is_ue8m0(KIND)) {
         // little-endian word of groups 4j..4j+3 assembled across the 4 groups'
-        // lanes (invalid groups contribute 0)
-        packed_word = ok ? (gs.e8 << (8u * (g & 3u))) : 0u;
-        packed_word |= __shfl_xor_sync(0xFFFFFFFFu, packed_word, L);
-        packed_word |= __shfl_xor_sync(0xFFFFFFFFu, packed_word, 2 * L);
+        // lanes (invalid groups contribute 0), for the layouts that store
+        // words; the fused kernels skip the two shuffles for the byte layouts
+        // (the plain ones keep them: the branch costs them registers)
+        if (!FUSED || p.layout == kPacked || p.layout == kTiled128x4) {   // warp-uniform
+            packed_word = ok ? (gs.e8 << (8u * (g & 3u))) : 0u;
+            packed_word |= __shfl_xor_sync(0xFFFFFFFFu, packed_word, L);
+            packed_word |= __shfl_xor_sync(0xFFFFFFFFu, packed_word, 2 * L);
+        }
     }
     if (!ok) return;
 
@@ -839,24 +929,34 @@ __device__ __forceinline__ void quantize_chunk(const Chunk<ITEMS, FUSED> &ch, co
 
 // Resident CTAs per SM the register allocation must allow (0: no constraint).
 // The fp32-scale plain variants run best at 5 (they take 46-48 registers; a
-// bound of 6 spills and was measured no better) and flat NVFP4 at 6 (<= 40
-// registers, no spills); the rest need no constraint.
+// bound of 6 spills and was measured no better), flat NVFP4 at 6 (<= 40
+// registers, no spills) and the fused ones at 8; the rest need no constraint.
 #ifndef PQG_MIN_BLOCKS_FP32
 #define PQG_MIN_BLOCKS_FP32 5
 #endif
 #ifndef PQG_MIN_BLOCKS_NVFP4
 #define PQG_MIN_BLOCKS_NVFP4 6
 #endif
-template <Kind KIND, bool FUSED, int DISP>
+// Fused kernels (4 warps per CTA) with one strip per chunk are held to 12
+// resident CTAs (40 registers; the short [4096, 2 x 2048] call 8.80 -> 8.71 us).
+// The 2-strip variants run best unbounded (65 registers, 7 CTAs): held to 8
+// CTAs they were slower ([4096, 2 x 7168] 25.09 -> 25.60 us).
+#ifndef PQG_MIN_BLOCKS_FUSED1
+#define PQG_MIN_BLOCKS_FUSED1 12
+#endif
+#ifndef PQG_MIN_BLOCKS_FUSED2
+#define PQG_MIN_BLOCKS_FUSED2 0
+#endif
+template <Kind KIND, bool FUSED, int DISP, int ITEMS>
 constexpr int min_blocks() {
-    if constexpr (FUSED) return 0;
+    if constexpr (FUSED) return ITEMS == 1 ? PQG_MIN_BLOCKS_FUSED1 : PQG_MIN_BLOCKS_FUSED2;
     if constexpr (KIND == Kind::E4M3_FP32 || KIND == Kind::INT8_FP32) return PQG_MIN_BLOCKS_FP32;
     if constexpr (KIND == Kind::E2M1_E4M3 && DISP == kFlat) return PQG_MIN_BLOCKS_NVFP4;
     return 0;
 }
 
 template <typename In, int G, Kind KIND, bool FUSED, int ITEMS, int WARPS, int DISP>
-__global__ void __launch_bounds__(WARPS * 32, min_blocks<KIND, FUSED, DISP>())
+__global__ void __launch_bounds__(WARPS * 32, min_blocks<KIND, FUSED, DISP, ITEMS>())
     quant_kernel(const __grid_constant__ Params p) {
     static_assert((G == 32 || G == 64 || G == 128) == (KIND != Kind::E2M1_E4M3) &&
                       (G == 16) == (KIND == Kind::E2M1_E4M3),
@@ -889,6 +989,10 @@ __global__ void __launch_bounds__(WARPS * 32, min_blocks<KIND, FUSED, DISP>())
         if (s >= t.total) break;                // warp-uniform
         Chunk<ITEMS, FUSED> ch;
         load_chunk<ITEMS, FUSED, DISP>(ch, s, min(items, t.total - s), t, p, lane);
+        if constexpr (PQG_PREFETCH_STRIP != 0) {
+            const uint32_t sn = s + gridDim.x * block;     // this warp's strips in its next block
+            if (sn < t.total) prefetch_chunk<ITEMS, FUSED, DISP>(sn, min(items, t.total - sn), t, p, lane);
+        }
         quantize_chunk<In, G, KIND, FUSED, ITEMS>(ch, p, lane, nv);
     }
     release_dependents();

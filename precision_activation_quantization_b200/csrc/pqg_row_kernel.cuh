@@ -23,6 +23,10 @@ namespace pqg {
 
 constexpr int kRowThreads = 256;  // 8 warps per CTA
 
+#ifndef PQG_PREFETCH_ROW
+#define PQG_PREFETCH_ROW 0
+#endif
+
 
 // The scale of row `row` of expert e.  One group per row: row-major,
 // column-major and packed all put it at element / word `row` of the expert's
@@ -89,6 +93,21 @@ __global__ void __launch_bounds__(kRowThreads)
                 }
             }
         }
+#if PQG_PREFETCH_ROW
+        // bring the row these warps take next into L2 while this one is
+        // reduced and encoded (one bulk prefetch of the whole row)
+        if (wr == 0) {                              // warp-uniform
+            const uint32_t rn = r + gridDim.x * rows_per_iter;
+            if (rn < t.total) {                     // warp-uniform
+                const Span sn = locate<VARLEN>(t, p.experts, rn);
+                const uint32_t rown = sn.base + (rn - sn.start);
+                if (lane == 0)
+                    prefetch_l2(p.in + sn.e * p.in_expert_bytes +
+                                    static_cast<uint64_t>(rown) * p.in_row_bytes,
+                                p.in_row_bytes);
+            }
+        }
+#endif
         // Fused rows keep silu(gate) * up in registers; plain rows keep the raw
         // 16-bit values (half the registers) and take the absmax on their
         // magnitude bits, widening only to quantize.
@@ -99,10 +118,7 @@ __global__ void __launch_bounds__(kRowThreads)
             for (int j = 0; j < SLOTS; ++j) {
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
-                    float g0, g1, u0, u1;
-                    widen2<In>(x[j][i], g0, g1);
-                    widen2<In>(u[j][i], u0, u1);
-                    const float2 y = silu_mul2(make_float2(g0, g1), make_float2(u0, u1));
+                    const float2 y = silu_mul_pair<In>(x[j][i], u[j][i]);
                     v[j][2 * i] = y.x;
                     v[j][2 * i + 1] = y.y;
                 }

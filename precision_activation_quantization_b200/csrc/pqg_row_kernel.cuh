@@ -23,8 +23,10 @@ namespace pqg {
 
 constexpr int kRowThreads = 256;  // 8 warps per CTA
 
+// Rows ahead of the current one that each row's first warp prefetches into L2
+// (0: none).  One row ahead took [8192, 7168] from 30.59 to 29.60 us.
 #ifndef PQG_PREFETCH_ROW
-#define PQG_PREFETCH_ROW 0
+#define PQG_PREFETCH_ROW 1
 #endif
 
 
@@ -94,10 +96,10 @@ __global__ void __launch_bounds__(kRowThreads)
             }
         }
 #if PQG_PREFETCH_ROW
-        // bring the row these warps take next into L2 while this one is
+        // bring a row these warps take later into L2 while this one is
         // reduced and encoded (one bulk prefetch of the whole row)
         if (wr == 0) {                              // warp-uniform
-            const uint32_t rn = r + gridDim.x * rows_per_iter;
+            const uint32_t rn = r + PQG_PREFETCH_ROW * gridDim.x * rows_per_iter;
             if (rn < t.total) {                     // warp-uniform
                 const Span sn = locate<VARLEN>(t, p.experts, rn);
                 const uint32_t rown = sn.base + (rn - sn.start);

@@ -90,9 +90,7 @@ inline int blocks_per_sm(OccupancyCache &cache, Kernel kernel, int device, int t
 #ifndef PQG_SHORT_WAVES
 #define PQG_SHORT_WAVES 4
 #endif
-#ifndef PQG_BALANCE_SHORT
-#define PQG_BALANCE_SHORT 0
-#endif
+
 
 // Fused multi-expert (masked) calls take 2 strips per chunk: they are long
 // enough for the deeper chunk to pay (masked 52.9 -> 51.5 us), while a short
@@ -166,18 +164,9 @@ cudaError_t launch_variant(const LaunchArgs &a) {
     if (a.expected_strips < wave * kWarps * kItems) p.items = 1;
     const uint64_t per_cta = static_cast<uint64_t>(kWarps) * p.items;
     uint64_t ctas = (a.expected_strips + per_cta - 1) / per_cta;
-    const bool short_call = ctas <= wave * PQG_SHORT_WAVES;
-    const uint64_t cap = short_call ? wave : wave * grid_waves<KIND, FUSED>(ctas, wave);
-    if (ctas > cap) {
-        if (PQG_BALANCE_SHORT && short_call) {
-            // as few CTAs as finish the blocks in the same number of rounds, so
-            // that the last round is not part-empty
-            const uint64_t rounds = (ctas + cap - 1) / cap;
-            ctas = (ctas + rounds - 1) / rounds;
-        } else {
-            ctas = cap;
-        }
-    }
+    const uint64_t cap =
+        ctas <= wave * PQG_SHORT_WAVES ? wave : wave * grid_waves<KIND, FUSED>(ctas, wave);
+    if (ctas > cap) ctas = cap;
     if (ctas < 1) ctas = 1;
 
     cudaLaunchConfig_t cfg = {};

@@ -58,6 +58,6 @@ def test_capture_commands_run_committed_code_on_known_workloads():
             assert flags[flags.index("--workload") + 1] in known, c
         assert set(f for f in flags if f.startswith("--")) <= {
             "--kernel-only", "--steps", "--warmup", "--no-cpu-baseline", "--workload",
-            "--samples"}, c
+            "--samples", "--gpus"}, c
         assert "--clock-control none" in c["ncu"], c
     assert len(caps) >= 9

@@ -747,58 +747,6 @@ __device__ __forceinline__ void load_chunk(Chunk<ITEMS, FUSED> &ch, uint32_t s, 
     }
 }
 
-// Prefetch into L2 the strips [s, s + n) a warp takes next (one bulk prefetch
-// per strip and half, issued by lane 0), so that their loads, issued after this
-// chunk's arithmetic, find them there.  Off: measured on looping grids it cost
-// the short fused call 19 % and the fp32-scale, FP4 and masked calls 4-12 %;
-// only the 65536-row fp16 INT8 sweep gained (2 %).
-#ifndef PQG_PREFETCH_STRIP
-#define PQG_PREFETCH_STRIP 0
-#endif
-template <int ITEMS, bool FUSED, int DISP>
-__device__ __forceinline__ void prefetch_chunk(uint32_t s, uint32_t n, const ExpertTable &t,
-                                               const Params &p, uint32_t lane) {
-    constexpr bool kVar = DISP == kVarlen;
-    uint32_t e = 0, start = 0, end_e = t.total, base = 0;
-    if constexpr (DISP != kFlat) {
-        const Span sp = locate<kVar>(t, p.experts, s);
-        e = sp.e;
-        start = sp.start;
-        end_e = sp.start + sp.strips;
-        base = sp.base;
-    }
-    uint32_t row = (s - start) / p.segs;
-    uint32_t seg = (s - start) - row * p.segs;
-#pragma unroll
-    for (int k = 0; k < ITEMS; ++k) {
-        if (static_cast<uint32_t>(k) >= n) break;      // warp-uniform
-        if constexpr (DISP != kFlat) {
-            if (s + k >= end_e) {
-                const Span sp = locate<kVar>(t, p.experts, s + k);
-                e = sp.e;
-                start = sp.start;
-                end_e = sp.start + sp.strips;
-                base = sp.base;
-                row = 0;
-                seg = 0;
-            }
-        }
-        if (lane == 0) {
-            const uint32_t col0 = seg * kStripElems;
-            const uint32_t bytes = min(kStripBytes, (p.K - col0) * 2u);
-            const uint8_t *src = p.in + e * p.in_expert_bytes +
-                                 static_cast<uint64_t>(base + row) * p.in_row_bytes +
-                                 static_cast<uint64_t>(col0) * 2u;
-            prefetch_l2(src, bytes);
-            if constexpr (FUSED) prefetch_l2(src + static_cast<uint64_t>(p.K) * 2u, bytes);
-        }
-        if (++seg == p.segs) {
-            seg = 0;
-            ++row;
-        }
-    }
-}
-
 // bf16 UE8M0 through the mixed-precision FMA path (1) or by widening (0).
 #ifndef PQG_UE8M0_MIXED
 #define PQG_UE8M0_MIXED 1
@@ -991,10 +939,6 @@ __global__ void __launch_bounds__(WARPS * 32, min_blocks<KIND, FUSED, DISP, ITEM
         if (s >= t.total) break;                // warp-uniform
         Chunk<ITEMS, FUSED> ch;
         load_chunk<ITEMS, FUSED, DISP>(ch, s, min(items, t.total - s), t, p, lane);
-        if constexpr (PQG_PREFETCH_STRIP != 0) {
-            const uint32_t sn = s + gridDim.x * block;     // this warp's strips in its next block
-            if (sn < t.total) prefetch_chunk<ITEMS, FUSED, DISP>(sn, min(items, t.total - sn), t, p, lane);
-        }
         quantize_chunk<In, G, KIND, FUSED, ITEMS>(ch, p, lane, nv);
     }
     release_dependents();

@@ -11,7 +11,6 @@
 #include <type_traits>
 
 #include "pqg_kernel.cuh"
-#include "pqg_pipe_kernel.cuh"
 #include "pqg_row_kernel.cuh"
 
 namespace pqg {
@@ -182,51 +181,6 @@ cudaError_t launch_variant(const LaunchArgs &a) {
     return cudaLaunchKernelEx(&cfg, kernel, p);
 }
 
-// Flat fused calls through the shared-memory pipelined kernel
-// (pqg_pipe_kernel.cuh): warps per CTA, strips per warp in the pipeline, and
-// the grid in waves of resident CTAs.
-#ifndef PQG_FUSED_PIPE
-#define PQG_FUSED_PIPE 0
-#endif
-#ifndef PQG_PIPE_WARPS
-#define PQG_PIPE_WARPS 4
-#endif
-#ifndef PQG_PIPE_STAGES
-#define PQG_PIPE_STAGES 2
-#endif
-#ifndef PQG_PIPE_WAVES
-#define PQG_PIPE_WAVES 1
-#endif
-
-template <typename In, int G, Kind KIND>
-cudaError_t launch_pipe(const LaunchArgs &a) {
-    constexpr int kWarps = PQG_PIPE_WARPS, kStages = PQG_PIPE_STAGES;
-    constexpr uint32_t kSmem = pipe_smem_bytes(kWarps, kStages);
-    auto kernel = fused_pipe_kernel<In, G, KIND, kWarps, kStages>;
-    int device = 0;
-    cudaError_t err = cudaGetDevice(&device);
-    if (err != cudaSuccess) return err;
-    static OccupancyCache cache;
-    const int bps = blocks_per_sm(cache, kernel, device, kWarps * 32, kSmem, kSmem);
-    const uint64_t wave = static_cast<uint64_t>(sm_count(device)) * bps;
-    uint64_t ctas = (a.expected_strips + kWarps - 1) / kWarps;
-    if (ctas > wave * PQG_PIPE_WAVES) ctas = wave * PQG_PIPE_WAVES;
-    if (ctas < 1) ctas = 1;
-    Params p = a.p;
-    p.items = 1;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(ctas), 1, 1);
-    cfg.blockDim = dim3(kWarps * 32, 1, 1);
-    cfg.dynamicSmemBytes = kSmem;
-    cfg.stream = a.stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = a.pdl ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, kernel, p);
-}
-
 template <typename In, int G, Kind KIND>
 cudaError_t launch_kind(const LaunchArgs &a) {
     if (a.disp == kVarlen)
@@ -235,7 +189,6 @@ cudaError_t launch_kind(const LaunchArgs &a) {
     const bool multi = a.p.experts > 1;
     if (a.fused) {
         if (multi) return launch_variant<In, G, KIND, true, kMasked>(a);
-        if constexpr (PQG_FUSED_PIPE != 0) return launch_pipe<In, G, KIND>(a);
         // A long flat fused call (4 or more waves of 1-strip work at 48 warps
         // per SM) runs a variant compiled for 2 strips per chunk: [4096, 2 x
         // 7168] 26.4 -> 24.6 us.  Short calls keep the 1-strip variant, whose

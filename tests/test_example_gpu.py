@@ -35,6 +35,15 @@ def test_usage_example_runs():
                        global_scale=g)
     assert tuple(q4.shape) == (1, 8192, 3584) and q4.dtype == torch.uint8
 
+    # grouped-contiguous MoE: 3 experts' tokens packed in segments padded to 128 rows
+    xp = torch.randn(384, 2 * 2048, device="cuda", dtype=torch.bfloat16)
+    indptr = torch.tensor([0, 128, 128, 384], device="cuda", dtype=torch.int32)
+    lens = torch.tensor([100, 0, 200], device="cuda", dtype=torch.int32)
+    q, s = pqg.quant_varlen(xp, indptr, lens, group=128, scale_fmt="ue8m0", layout="col",
+                            fuse_silu_mul=True)
+    assert tuple(q.shape) == (384, 2048) and q.dtype == torch.float8_e4m3fn
+    assert tuple(s.shape) == (16, 384)
+
     # fused SiLU-and-mul over [gate | up] rows, masked MoE dispatch
     h = torch.randn(32, 2048, 2 * 2048, device="cuda", dtype=torch.bfloat16)
     masked_m = torch.randint(0, 2049, (32,), device="cuda", dtype=torch.int32)

@@ -81,6 +81,20 @@ bool overlaps(const void *a, int64_t na, const void *b, int64_t nb) {
 }  // namespace
 
 namespace pqg {
+// magic and shift of div_segs (pqg_kernel.cuh): l = ceil(log2 segs),
+// magic = ceil(2^(31 + l) / segs), shift = l - 1; segs == 1 gives magic 0.
+void segs_divider(uint32_t segs, uint32_t *magic, uint32_t *shift) {
+    if (segs <= 1u) {
+        *magic = 0u;
+        *shift = 0u;
+        return;
+    }
+    uint32_t l = 0;
+    while ((1ull << l) < segs) ++l;
+    *magic = static_cast<uint32_t>(((1ull << (31u + l)) + segs - 1u) / segs);
+    *shift = l - 1u;
+}
+
 int sm_count(int device) {
     if (device < 0 || device >= kMaxDevices) device = 0;
     int n = g_sm_count[device].load(std::memory_order_relaxed);
@@ -173,6 +187,7 @@ int quant_impl(const void *in, void *out, void *scales, const float *global_scal
     a.p.in_row_bytes = static_cast<uint32_t>(in_row_bytes);
     a.p.ng = static_cast<uint32_t>(K / group);
     a.p.segs = static_cast<uint32_t>((K + pqg::kStripElems - 1) / pqg::kStripElems);
+    pqg::segs_divider(a.p.segs, &a.p.segs_magic, &a.p.segs_shift);
     a.p.mpad = static_cast<uint32_t>(padded_rows(M));
     a.p.layout = static_cast<uint32_t>(scale_layout);
     a.p.experts = static_cast<uint32_t>(num_experts);

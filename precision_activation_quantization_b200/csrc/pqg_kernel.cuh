@@ -121,6 +121,8 @@ struct Params {
     uint32_t out_row_bytes;    // K (one byte per code) or K/2 (E2M1, two per byte)
     uint32_t ng;               // groups per row
     uint32_t segs;             // strips per row = ceil(K / 512)
+    uint32_t segs_magic;       // s / segs = umulhi(s, segs_magic) >> segs_shift (0: segs == 1)
+    uint32_t segs_shift;
     uint32_t mpad;             // rows of a column-major plane (M rounded up to 4)
     uint32_t layout;           // kRowMajor / kColMajor / kPacked
     uint32_t experts;          // <= kMaxExperts
@@ -368,6 +370,18 @@ __device__ __forceinline__ uint32_t absmax_bits16(const uint32_t (&w)[8]) {
     uint32_t b = __vimax3_u16x2(m[3], m[4], m[5]);
     a = __vimax3_u16x2(a, b, __vimax3_u16x2(m[6], m[7], 0u));
     return max(a & 0xFFFFu, a >> 16);
+}
+
+// max |v| over 16 values as a tree (depth 4 instead of a chain of 16)
+__device__ __forceinline__ float absmax16(const float (&v)[16]) {
+    float m[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) m[i] = fmaxf(fabsf(v[2 * i]), fabsf(v[2 * i + 1]));
+#pragma unroll
+    for (int w = 4; w >= 1; w >>= 1)
+#pragma unroll
+        for (int i = 0; i < w; ++i) m[i] = fmaxf(m[i], m[i + w]);
+    return m[0];
 }
 
 // The value of a non-negative finite bf16 / fp16 magnitude pattern (the
@@ -679,6 +693,17 @@ __device__ __forceinline__ Span locate(const ExpertTable &t, uint32_t experts, u
     return sp;
 }
 
+// s / segs for s < 2^31 without a division instruction sequence (which costs
+// about twenty instructions and an SFU operation per call): with l =
+// ceil(log2 segs) >= 1, magic = ceil(2^(31 + l) / segs) < 2^32 and shift = l - 1,
+// the quotient is umulhi(s, magic) >> shift.  Exact for every s < 2^31 because
+// magic * segs - 2^(31 + l) < segs <= 2^l (Granlund and Montgomery, "Division by
+// invariant integers using multiplication", PLDI 1994, Theorem 4.2, with N = 31).
+// segs == 1 has magic 0 and returns s.  The host computes magic and shift.
+__device__ __forceinline__ uint32_t div_segs(uint32_t s, const Params &p) {
+    return p.segs_magic == 0u ? s : (__umulhi(s, p.segs_magic) >> p.segs_shift);
+}
+
 // ---------------------------------------------------------------------------
 // One chunk of up to ITEMS strips held in registers
 // ---------------------------------------------------------------------------
@@ -708,7 +733,7 @@ __device__ __forceinline__ void load_chunk(Chunk<ITEMS, FUSED> &ch, uint32_t s, 
         end_e = sp.start + sp.strips;
         base = sp.base;
     }
-    uint32_t row = (s - start) / p.segs;
+    uint32_t row = div_segs(s - start, p);
     uint32_t seg = (s - start) - row * p.segs;
 #pragma unroll
     for (int k = 0; k < ITEMS; ++k) {
@@ -806,9 +831,7 @@ __device__ __forceinline__ void quantize_strip(const uint32_t (&x)[8], const uin
                 widen2<In>(x[i], v[2 * i], v[2 * i + 1]);
             }
         }
-        float amax = 0.0f;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
+        float amax = absmax16(v);
 #pragma unroll
         for (int o = 1; o < L; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
         gs = make_scale<KIND>(amax, nv);

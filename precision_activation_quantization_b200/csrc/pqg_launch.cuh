@@ -29,6 +29,7 @@ struct LaunchArgs {
 };
 
 int sm_count(int device);  // cached cudaDevAttrMultiProcessorCount
+void segs_divider(uint32_t segs, uint32_t *magic, uint32_t *shift);
 
 // Resident CTAs per SM of one kernel variant, cached per device: the
 // occupancy query (and the shared-memory attribute it needs) applies to the
@@ -260,6 +261,8 @@ cudaError_t launch_row_variant(const LaunchArgs &a, uint32_t wpr) {
 
     Params p = a.p;
     p.segs = 1;        // the expert table counts rows
+    p.segs_magic = 0;  // (no strip division)
+    p.segs_shift = 0;
     p.items = wpr;     // warps per row
     const uint64_t rows_per_cta = (kRowThreads / 32) / wpr;
     uint64_t ctas = (a.expected_rows + rows_per_cta - 1) / rows_per_cta;

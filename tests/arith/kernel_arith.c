@@ -24,6 +24,13 @@
  *                        that can give a nonzero code; kind 0 = E4M3 (the
  *                        quotient carried negated, as the kernel does), 1 = INT8.
  *
+ *   divsegs              s / segs by umulhi(s, magic) >> shift with l =
+ *                        ceil(log2 segs), magic = ceil(2^(31+l) / segs), shift =
+ *                        l - 1 (segs == 1: s itself), against the division, for
+ *                        every segs up to 2^20 and, per segs, the s < 2^31 next to
+ *                        every quotient boundary at both ends of the range plus
+ *                        pseudo-random s.
+ *
  * A last argument <stride> > 1 checks every stride-th case only.  Build:
  * gcc -O2 -mfma -fopenmp -ffp-contract=off kernel_arith.c -lm
  * (fmaf must be a true fused multiply-add; -ffp-contract=off keeps every
@@ -174,6 +181,37 @@ int main(int argc, char **argv) {
                     ++n;
                     bad += !same;
                 }
+            }
+        }
+    } else if (!strcmp(argv[1], "divsegs")) {
+        const long long stride = argc > 2 ? atoll(argv[2]) : 1;
+#pragma omp parallel for schedule(dynamic, 256) reduction(+ : bad, n)
+        for (long long d = 1; d <= (1ll << 20); d += stride) {
+            uint32_t magic = 0, shift = 0;
+            if (d > 1) {
+                uint32_t l = 0;
+                while ((1ull << l) < (unsigned long long)d) ++l;
+                magic = (uint32_t)(((1ull << (31u + l)) + (unsigned long long)d - 1u) / (unsigned long long)d);
+                shift = l - 1u;
+            }
+            const uint32_t top = 0x7FFFFFFFu;
+            uint64_t x = 0x9E3779B97F4A7C15ull ^ (uint64_t)d;
+            for (int i = 0; i < 200; ++i) {
+                uint32_t s;
+                if (i < 64) {                        /* around the lowest boundaries */
+                    s = (uint32_t)((i / 2) * d + (i % 2 ? d - 1 : 0));
+                } else if (i < 128) {                /* around the highest ones */
+                    const uint64_t k = top / (uint64_t)d - (uint64_t)((i - 64) / 2);
+                    const uint64_t v = k * (uint64_t)d + ((i % 2) ? (uint64_t)d - 1 : 0);
+                    s = (uint32_t)(v > top ? top : v);
+                } else {                             /* pseudo-random */
+                    x ^= x << 13; x ^= x >> 7; x ^= x << 17;
+                    s = (uint32_t)(x & top);
+                }
+                const uint32_t q = magic == 0u ? s
+                                   : (uint32_t)(((uint64_t)s * magic) >> 32) >> shift;
+                ++n;
+                bad += q != s / (uint32_t)d;
             }
         }
     } else {

@@ -7,7 +7,8 @@ every shortcut in plain C and compares it with the definition it replaces):
 - the UE8M0 byte from the exponent and mantissa bits of amax, with no
   division (FMAX 448 and FMAX 6);
 - RN(amax / c) for c = 448, 127 and 6 by a reciprocal and two Markstein steps;
-- one Markstein step (instead of two) before the E4M3 / INT8 cast of x / s.
+- one Markstein step (instead of two) before the E4M3 / INT8 cast of x / s;
+- s / segs (strip index to row) by a multiply-high with a host-computed magic.
 
 By default every 97th (or 4099th) case is checked, so the suite stays fast;
 ``PQG_EXHAUSTIVE=1`` checks every case (minutes on 8 cores for bf16, about half
@@ -65,3 +66,10 @@ def test_one_markstein_step_near_every_rounding_midpoint(checker, bits, kind):
     """The cases that can fail: x / s within a few ulps of a code midpoint."""
     n, bad = run(checker, "hard", bits, kind)
     assert n > 500_000 and bad == 0
+
+
+def test_strip_row_division_by_magic_multiply(checker):
+    """Every strips-per-row count up to 2^20 (K up to 2^29), 200 strip indices
+    each: both ends of the index range next to quotient boundaries, and random."""
+    n, bad = run(checker, "divsegs", 1)
+    assert n == 200 * (1 << 20) and bad == 0

@@ -1,5 +1,5 @@
-// Instantiates the bf16-input half of the kernel family (65 strip-kernel and
-// 18 per-token variants).
+// Instantiates the bf16-input half of the kernel family (91 strip-kernel and
+// 36 per-token variants).
 #include "pqg_launch.cuh"
 
 namespace pqg {

@@ -159,7 +159,10 @@ enum pqg_scale_layout {
  *          device, so it may be produced by the preceding kernel on `stream`.
  * expected_m  a hint for the masked grid: the typical masked_m value.  Results
  *          never depend on it; <= 0 or > M means M.  Ignored when masked_m is
- *          NULL.
+ *          NULL.  A fused masked call with at most 32 experts and
+ *          1 <= expected_m <= 8 (decode) reads each expert's first
+ *          min(expected_m, M) input rows while masked_m is still in flight;
+ *          rows past masked_m among them are read but never written.
  * stream   CUDA stream the kernel is launched on.  The launch carries the
  *          programmatic-dependent-launch attribute (see pqg_set_pdl); the kernel
  *          waits for the preceding grid before its first global-memory access.

@@ -25,6 +25,7 @@ std::atomic<int> g_sm_count[kMaxDevices];
 int64_t padded_rows(int64_t M) { return (M + 3) / 4 * 4; }
 
 constexpr int64_t kMaxPerTokenK = 16384;
+constexpr int64_t kMaxSpecRows = 8;   // expected_m up to which masked calls load rows speculatively
 
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
@@ -209,6 +210,19 @@ int quant_impl(const void *in, void *out, void *scales, const float *global_scal
              : out_dtype == PQG_INT8        ? pqg::Kind::INT8_FP32
                                             : pqg::Kind::E4M3_FP32;
     a.disp = varlen ? pqg::kVarlen : num_experts > 1 ? pqg::kMasked : pqg::kFlat;
+    // Small fused masked calls (decode: a few rows per expert, at most 32
+    // experts) load each expert's first expected_m rows without waiting for
+    // masked_m (pqg_kernel.cuh, kMaskedSpec); rows past masked_m are read there
+    // but never written.
+    a.p.spec = 0;
+    a.p.spec_magic = 0;
+    a.p.spec_shift = 0;
+    if (a.disp == pqg::kMasked && masked_m != nullptr && fuse_silu_mul != 0 && num_experts <= 32 &&
+        expected_m >= 1 && expected_m <= kMaxSpecRows) {
+        a.disp = pqg::kMaskedSpec;
+        a.p.spec = static_cast<uint32_t>(std::min(expected_m, M));
+        pqg::segs_divider(a.p.spec * a.p.segs, &a.p.spec_magic, &a.p.spec_shift);
+    }
     a.fused = fuse_silu_mul != 0;
     a.pdl = g_pdl.load(std::memory_order_relaxed) != 0;
     a.stream = reinterpret_cast<cudaStream_t>(stream);

@@ -127,13 +127,16 @@ struct Params {
     uint32_t layout;           // kRowMajor / kColMajor / kPacked
     uint32_t experts;          // <= kMaxExperts
     uint32_t items;            // strips per warp per block, 1 .. ITEMS
+    uint32_t spec;             // kMaskedSpec: rows per expert loaded before masked_m is known
+    uint32_t spec_magic;       // s / (spec * segs), as segs_magic
+    uint32_t spec_shift;
 };
 
 // Dispatch forms: one expert's M rows (flat), E experts of M rows each with a
 // per-expert row count (masked), or E segments of one buffer of M packed rows
 // (varlen, grouped-contiguous: expert strides are 0 and a segment's rows
 // start at its own row offset).
-enum : int { kFlat = 0, kMasked = 1, kVarlen = 2 };
+enum : int { kFlat = 0, kMasked = 1, kVarlen = 2, kMaskedSpec = 3 };
 
 // Dynamic shared memory of one CTA: the expert prefix table (more than 32
 // experts only), followed by the segments' first rows when varlen.
@@ -723,7 +726,7 @@ template <int ITEMS, bool FUSED, int DISP>
 __device__ __forceinline__ void load_chunk(Chunk<ITEMS, FUSED> &ch, uint32_t s, uint32_t n,
                                            const ExpertTable &t, const Params &p,
                                            uint32_t lane) {
-    constexpr bool kVar = DISP == kVarlen;
+    constexpr bool kVar = DISP == kVarlen || DISP == kMaskedSpec;   // the table holds first rows
     ch.n = n;
     uint32_t e = 0, start = 0, end_e = t.total, base = 0;
     if constexpr (DISP != kFlat) {
@@ -768,6 +771,49 @@ __device__ __forceinline__ void load_chunk(Chunk<ITEMS, FUSED> &ch, uint32_t s, 
         if (++seg == p.segs) {
             seg = 0;
             ++row;
+        }
+    }
+}
+
+// The speculative region of a small masked call (kMaskedSpec, at most 32
+// experts): the first p.spec rows of every expert, strips in (expert, row,
+// strip-in-row) order, loaded without waiting for masked_m.  Every address
+// lies inside the expert's M rows (spec <= M); whether a row is live is
+// decided after the loads, and dead rows are neither quantized nor written.
+template <int ITEMS, bool FUSED>
+__device__ __forceinline__ void load_spec_chunk(Chunk<ITEMS, FUSED> &ch, uint32_t s, uint32_t n,
+                                                const Params &p, uint32_t lane) {
+    ch.n = n;
+    const uint32_t per_e = p.spec * p.segs;
+    uint32_t e = p.spec_magic == 0u ? s : (__umulhi(s, p.spec_magic) >> p.spec_shift);
+    const uint32_t r = s - e * per_e;
+    uint32_t row = div_segs(r, p);
+    uint32_t seg = r - row * p.segs;
+#pragma unroll
+    for (int k = 0; k < ITEMS; ++k) {
+        const bool live = static_cast<uint32_t>(k) < n;
+        ch.e[k] = e;
+        ch.row[k] = row;
+        ch.col[k] = seg * kStripElems + lane * 16u;
+        if (live && ch.col[k] < p.K) {
+            const uint8_t *src = p.in + e * p.in_expert_bytes +
+                                 static_cast<uint64_t>(row) * p.in_row_bytes +
+                                 static_cast<uint64_t>(ch.col[k]) * 2u;
+            load32B(src, ch.x[k]);
+            if constexpr (FUSED) load32B(src + static_cast<uint64_t>(p.K) * 2u, ch.u[k]);
+        } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                ch.x[k][i] = 0u;
+                if constexpr (FUSED) ch.u[k][i] = 0u;
+            }
+        }
+        if (++seg == p.segs) {
+            seg = 0;
+            if (++row == p.spec) {
+                row = 0;
+                ++e;
+            }
         }
     }
 }
@@ -943,7 +989,45 @@ __global__ void __launch_bounds__(WARPS * 32, min_blocks<KIND, FUSED, DISP, ITEM
     const uint32_t warp = threadIdx.x >> 5;
     if constexpr (KIND == Kind::E2M1_E4M3) build_nvfp4_table(p, nv);
     ExpertTable t;
-    if constexpr (DISP != kFlat) {
+    if constexpr (DISP == kMaskedSpec) {
+        // Small masked calls (decode): the rows every expert is expected to
+        // have are loaded at once, in parallel with masked_m, instead of after
+        // it; the rest of each expert's rows follow through the warp table.
+        uint32_t live_rows = 0;                 // lane e: rows of expert e (E <= 32)
+        if (lane < p.experts)
+            live_rows = static_cast<uint32_t>(
+                min(max(__ldg(p.masked_m + lane), 0), static_cast<int>(p.M)));
+        const uint32_t items = p.items, block = WARPS * items;
+        const uint32_t total_spec = p.experts * p.spec * p.segs;
+        const uint32_t nblocks_spec = (total_spec + block - 1) / block;
+        for (uint32_t blk = blockIdx.x; blk < nblocks_spec; blk += gridDim.x) {
+            const uint32_t s = blk * block + warp * items;
+            if (s >= total_spec) break;         // warp-uniform
+            Chunk<ITEMS, FUSED> ch;
+            load_spec_chunk<ITEMS, FUSED>(ch, s, min(items, total_spec - s), p, lane);
+#pragma unroll
+            for (int k = 0; k < ITEMS; ++k) {
+                if (static_cast<uint32_t>(k) >= ch.n) break;   // warp-uniform
+                const uint32_t rows = __shfl_sync(0xFFFFFFFFu, live_rows, ch.e[k]);
+                if (ch.row[k] < rows)           // warp-uniform
+                    quantize_strip<In, G, KIND, FUSED>(ch.x[k], FUSED ? ch.u[k] : nullptr,
+                                                       ch.e[k], ch.row[k], ch.col[k], p, lane, nv);
+            }
+        }
+        // rows [spec, live) of each expert: a warp table whose first row is spec
+        t.mode = 1;
+        t.prefix = nullptr;
+        t.base = p.spec;
+        t.cnt = lane < p.experts && live_rows > p.spec ? (live_rows - p.spec) * p.segs : 0u;
+        uint32_t incl = t.cnt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+            if (lane >= static_cast<uint32_t>(o)) incl += v;
+        }
+        t.incl = incl;
+        t.total = __shfl_sync(0xFFFFFFFFu, incl, 31);
+    } else if constexpr (DISP != kFlat) {
         t = make_table<DISP == kVarlen>(p, smem_prefix, lane);
     } else {
         uint32_t first;

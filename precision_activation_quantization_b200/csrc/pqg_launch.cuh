@@ -22,7 +22,7 @@ struct LaunchArgs {
     uint64_t expected_rows;    // rows the grid is sized for (per-token kernel)
     int group;                 // 32 / 64 / 128, or K (per-token)
     Kind kind;
-    int disp;                  // kFlat, kMasked or kVarlen
+    int disp;                  // kFlat, kMasked, kVarlen or kMaskedSpec
     bool fused;
     bool pdl;
     cudaStream_t stream;
@@ -187,6 +187,8 @@ cudaError_t launch_kind(const LaunchArgs &a) {
     if (a.disp == kVarlen)
         return a.fused ? launch_variant<In, G, KIND, true, kVarlen>(a)
                        : launch_variant<In, G, KIND, false, kVarlen>(a);
+    if (a.disp == kMaskedSpec)   // fused only (chosen by the caller)
+        return launch_variant<In, G, KIND, true, kMaskedSpec>(a);
     const bool multi = a.p.experts > 1;
     if (a.fused) {
         if (multi) return launch_variant<In, G, KIND, true, kMasked>(a);

@@ -1,4 +1,4 @@
-// Instantiates the bf16-input half of the kernel family (91 strip-kernel and
+// Instantiates the bf16-input half of the kernel family (104 strip-kernel and
 // 36 per-token variants).
 #include "pqg_launch.cuh"
 

@@ -400,6 +400,46 @@ def test_per_token_full_size():
 # --------------------------------------------------------------------------
 
 # --------------------------------------------------------------------------
+# small fused masked calls: the first expected_m rows loaded before masked_m
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("kind", [("e4m3", "ue8m0", "col"), ("e4m3", "fp32", "row"),
+                                  ("int8", "fp32", "col"), ("e2m1", "ue8m0", "tile128x4")],
+                         ids=lambda k: "_".join(k))
+@pytest.mark.parametrize("E,M,expected_m", [(32, 6, 1), (32, 16, 2), (2, 40, 8), (17, 5, 8),
+                                            (3, 3, 7)])
+def test_masked_speculative_rows(kind, E, M, expected_m):
+    """Fused masked calls with expected_m <= 8 and at most 32 experts read each
+    expert's first min(expected_m, M) rows before masked_m is known: live rows
+    match the oracle, dead rows (read, never written) keep the sentinel, and
+    rows past expected_m of the larger experts are covered too."""
+    rng = np.random.default_rng(E * 100 + M + expected_m)
+    mm = rng.integers(-2, M + 3, size=E).astype(np.int32)
+    mm[0] = M                                     # one full expert, one empty
+    mm[-1] = 0
+    for K, G in ((640, 128), (1536, 32)):
+        w = make(M, K, G, kind, fused=True, E=E, seed=int(mm.sum()) + K, masked_m=mm,
+                 expected_m=expected_m)
+        check_fused(w, max_flip_frac=1e-3)
+
+
+def test_unmasked_experts_ignore_small_expected_m():
+    """Without masked_m every expert's M rows are quantized; a small expected_m
+    (ignored there) must not send the call down the speculative masked path."""
+    for E, M, expected_m in ((4, 9, 1), (32, 3, 8)):
+        w = make(M, 1024, 128, ("e4m3", "ue8m0", "col"), fused=True, E=E, seed=E + M,
+                 expected_m=expected_m)
+        check_fused(w, max_flip_frac=1e-3)
+
+
+def test_masked_decode_nvfp4_speculative():
+    E, M = 32, 4
+    mm = np.random.default_rng(7).integers(0, 2, size=E).astype(np.int32)
+    check_fused(make_nv(M, 512, 2.625, "tile128x4", fused=True, E=E, seed=8, masked_m=mm,
+                        expected_m=1), max_flip_frac=1e-3)
+
+
+# --------------------------------------------------------------------------
 # grouped-contiguous (varlen): token segments packed in one buffer
 # --------------------------------------------------------------------------
 

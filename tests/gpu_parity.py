@@ -175,8 +175,8 @@ def _log_flips(w, flips, n_el, scale_flips, budget):
 
 
 def check_fused(w, *, max_flip_frac=CONTRACT_FLIP_FRAC, rel_tol=7e-2, **kw):
-    """Fused contract: UE8M0 bytes equal unless the oracle's amax/448 is within
-    2^-20 of a power of two; fp32 scales within 2^-19 relative; codes equal
+    """Fused contract: UE8M0 bytes equal unless the oracle's amax/FMAX (448 for
+    E4M3, 6 for E2M1) is within 2^-20 of a power of two; fp32 scales within 2^-19 relative; codes equal
     except for at most ``max_flip_frac`` of elements (outside groups whose UE8M0
     exponent flipped), each moving by one step; every element's dequantized
     value within ``rel_tol`` of the oracle's silu(gate)*up."""
@@ -245,7 +245,8 @@ def check_fused(w, *, max_flip_frac=CONTRACT_FLIP_FRAC, rel_tol=7e-2, **kw):
     elif g_e8 is not None:
         g_e8, r_e8 = g_e8[live].astype(np.int64), r_e8[live].astype(np.int64)
         scale_diff = g_e8 != r_e8
-        r = (amax[live] / 448.0)
+        # the byte is the exponent of amax / FMAX: 448 for E4M3, 6 for E2M1 (MXFP4)
+        r = amax[live] / (6.0 if w.out_dtype == "e2m1" else 448.0)
         near_pow2 = np.abs(r / np.exp2(np.round(np.log2(r))) - 1.0) < 2.0 ** -20
         assert (~scale_diff | near_pow2).all(), \
             f"{w.name}: {int((scale_diff & ~near_pow2).sum())} UE8M0 bytes differ away from a power of two"

@@ -122,6 +122,44 @@ def test_fused_check_catches_a_moved_ue8m0_byte(monkeypatch):
         check_fused(_fp8_fused())
 
 
+def _mxfp4_tie_group(up_bits):
+    """A fused MXFP4 call (G = 32, row-major UE8M0) whose expert 0, row 0,
+    group 0 has every gate 64 (sigmoid(64) is 1 in fp64) and every up the bf16
+    value up_bits, so that each of its 32 elements is 64 * up."""
+    w = make(M, K, 32, ("e2m1", "ue8m0", "row"), fused=True, E=E, seed=5, masked_m=MASK)
+    x = w.x.reshape(E, M, 2 * K)
+    x[0, 0, :32] = 0x4280                            # bf16 64.0
+    x[0, 0, K:K + 32] = up_bits
+    return w
+
+
+def _rescaled_group(w, q, s):
+    """The group quantized as a device whose amax came out one ulp high would:
+    its UE8M0 byte one higher and every code E2M1 3 (6 at the halved scale)."""
+    assert s[0] == 127 and (q[:16] == 0x77).all()   # oracle: 2^0 and all codes 6
+    s[0] += 1
+    q[:16] = 0x55
+
+
+def test_fused_check_allows_an_mxfp4_byte_flip_at_a_power_of_two(monkeypatch):
+    """MXFP4 takes the exponent of amax / 6: amax = 6 * 2^0 sits on a power of
+    two, so the byte may move by one (with the group's codes rescaled)."""
+    w = _mxfp4_tie_group(0x3DC0)                     # up = 0.09375: 64 * up = 6 exactly
+    _device_returns(monkeypatch, _rescaled_group)
+    assert check_fused(w, max_flip_frac=1e-3)["scale_flips"] == 1
+
+
+def test_fused_check_rejects_an_mxfp4_byte_flip_away_from_a_power_of_two(monkeypatch):
+    w = _mxfp4_tie_group(0x3DCD)                     # up = 0.10009765625: amax / 6 = 1.0677
+
+    def bump(w, q, s):
+        s[0] += 1
+        q[:16] = 0x55
+    _device_returns(monkeypatch, bump)
+    with pytest.raises(AssertionError, match="away from a power of two"):
+        check_fused(w, max_flip_frac=1e-3)
+
+
 def test_fused_check_catches_an_fp32_scale_off_by_2_to_minus_10(monkeypatch):
     def scale(w, q, s):
         f = s.view(np.float32)

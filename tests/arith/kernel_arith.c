@@ -24,14 +24,15 @@
  *                        that can give a nonzero code; kind 0 = E4M3 (the
  *                        quotient carried negated, as the kernel does), 1 = INT8.
  *
- *   divsegs              s / segs by umulhi(s, magic) >> shift with l =
+ *   divsegs [<stride> <dmin> <dmax>]
+ *                        s / segs by umulhi(s, magic) >> shift with l =
  *                        ceil(log2 segs), magic = ceil(2^(31+l) / segs), shift =
  *                        l - 1 (segs == 1: s itself), against the division, for
- *                        every segs up to 2^20 and, per segs, the s < 2^31 next to
- *                        every quotient boundary at both ends of the range plus
- *                        pseudo-random s.
+ *                        every segs in [dmin, dmax] (default 1 .. 2^20) and, per
+ *                        segs, the s < 2^31 next to every quotient boundary at
+ *                        both ends of the range plus pseudo-random s.
  *
- * A last argument <stride> > 1 checks every stride-th case only.  Build:
+ * A <stride> > 1 checks every stride-th case only.  Build:
  * gcc -O2 -mfma -fopenmp -ffp-contract=off kernel_arith.c -lm
  * (fmaf must be a true fused multiply-add; -ffp-contract=off keeps every
  * other operation rounded on its own).
@@ -185,8 +186,10 @@ int main(int argc, char **argv) {
         }
     } else if (!strcmp(argv[1], "divsegs")) {
         const long long stride = argc > 2 ? atoll(argv[2]) : 1;
+        const long long dmin = argc > 3 ? atoll(argv[3]) : 1;
+        const long long dmax = argc > 4 ? atoll(argv[4]) : (1ll << 20);
 #pragma omp parallel for schedule(dynamic, 256) reduction(+ : bad, n)
-        for (long long d = 1; d <= (1ll << 20); d += stride) {
+        for (long long d = dmin; d <= dmax; d += stride) {
             uint32_t magic = 0, shift = 0;
             if (d > 1) {
                 uint32_t l = 0;

@@ -8,7 +8,8 @@ every shortcut in plain C and compares it with the definition it replaces):
   division (FMAX 448 and FMAX 6);
 - RN(amax / c) for c = 448, 127 and 6 by a reciprocal and two Markstein steps;
 - one Markstein step (instead of two) before the E4M3 / INT8 cast of x / s;
-- s / segs (strip index to row) by a multiply-high with a host-computed magic.
+- s / segs (strip index to row), and s / (spec * segs) in the masked decode
+  form, by a multiply-high with a host-computed magic.
 
 By default every 97th (or 4099th) case is checked, so the suite stays fast;
 ``PQG_EXHAUSTIVE=1`` checks every case (minutes on 8 cores for bf16, about half
@@ -73,3 +74,10 @@ def test_strip_row_division_by_magic_multiply(checker):
     each: both ends of the index range next to quotient boundaries, and random."""
     n, bad = run(checker, "divsegs", 1)
     assert n == 200 * (1 << 20) and bad == 0
+
+
+def test_decode_region_division_by_magic_multiply(checker):
+    """The masked decode form divides by spec * segs (spec <= 8, segs <= 2^19):
+    every divisor from 2^20 + 1 to 2^22, 200 strip indices each."""
+    n, bad = run(checker, "divsegs", 1, (1 << 20) + 1, 1 << 22)
+    assert n == 200 * 3 * (1 << 20) and bad == 0

@@ -423,6 +423,18 @@ def test_masked_speculative_rows(kind, E, M, expected_m):
         check_fused(w, max_flip_frac=1e-3)
 
 
+@pytest.mark.parametrize("kind", [("e4m3", "ue8m0", "packed"), ("int8", "fp32", "row")],
+                         ids=lambda k: "_".join(k))
+def test_masked_speculative_rows_fp16(kind):
+    """The decode form with fp16 input: live rows match the oracle, dead rows
+    keep the sentinel."""
+    E, M, expected_m = 32, 12, 4
+    mm = np.random.default_rng(41).integers(-1, 10, size=E).astype(np.int32)
+    w = make(M, 1152, 64, kind, in_dtype="fp16", fused=True, E=E, seed=42, masked_m=mm,
+             expected_m=expected_m)
+    check_fused(w, max_flip_frac=1e-3)
+
+
 def test_unmasked_experts_ignore_small_expected_m():
     """Without masked_m every expert's M rows are quantized; a small expected_m
     (ignored there) must not send the call down the speculative masked path."""

@@ -51,6 +51,10 @@ MUTANTS = {
                                   "float x = pqgo_decode(xrow[(fused ? K : 0) + b * G + i], in_fp16);"),
     "silu_wrong_sign": ("double silu = g / (1.0 + exp(-g));",
                         "double silu = g / (1.0 + exp(g));"),
+    "silu_single_precision": ("double silu = g / (1.0 + exp(-g));",
+                              "double silu = (float)g / (1.0f + expf(-(float)g));"),
+    "silu_product_rounded_twice": ("return (float)(silu * (double)up);",
+                                   "return (float)((float)silu * (float)up);"),
     "packed_padding_not_zeroed": ("((uint8_t *)scales)[word * 4 + b] = 0;", ";"),
     "fp16_subnormal_exponent": ("v = ldexp((double)m, -24);", "v = ldexp((double)m, -25);"),
     "int8_truncates": ("double n = nearbyint((double)t);", "double n = trunc((double)t);"),

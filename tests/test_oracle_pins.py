@@ -596,6 +596,38 @@ def test_silu_mul_matches_torch_float64():
     assert (ulp == 0).mean() > 0.99999
 
 
+def test_silu_mul_is_correctly_rounded_against_long_double():
+    """P-9 in its stated form: silu(g) * u evaluated independently, in 80-bit
+    long double and through sigmoid(g) = exp(-log1p(exp(-g))), then rounded once
+    to fp32.  The oracle (double, one rounding) must give exactly that value,
+    signed zeros and subnormal results included, except where the exact product
+    lies within 2^-40 relative of an fp32 rounding midpoint (double's own error,
+    about 2^-50, could cross it there)."""
+    assert np.finfo(np.longdouble).nmant >= 63, "needs x87 extended long double"
+    rng = np.random.default_rng(61)
+    g = np.concatenate([rng.standard_normal(200_000).astype(np.float32) * 4,
+                        (rng.standard_normal(50_000) * 40).astype(np.float32),
+                        np.float32([0.0, -0.0, 1e-30, -1e-30, 30.0, -30.0, 88.0, -88.0,
+                                    100.0, -100.0])])
+    u = rng.standard_normal(g.size).astype(np.float32)
+    u[-10:] = np.float32([1.0, 1.0, 2.0, -0.5, 1.0, 1.0, -3.0, 1.0, 0.25, -1.0])
+    gl, ul = g.astype(np.longdouble), u.astype(np.longdouble)
+    exact = gl * np.exp(-np.log1p(np.exp(-gl))) * ul
+    want = exact.astype(np.float32)
+    got = oracle.silu_mul(g, u)
+    up = np.nextafter(want, np.float32(np.inf)).astype(np.longdouble)
+    dn = np.nextafter(want, np.float32(-np.inf)).astype(np.longdouble)
+    w = want.astype(np.longdouble)
+    gap = np.minimum(np.abs(exact - (w + up) / 2), np.abs(exact - (w + dn) / 2))
+    with np.errstate(divide="ignore", invalid="ignore"):
+        near_tie = (exact != 0) & (gap / np.abs(exact) < np.longdouble(2.0) ** -40)
+    assert near_tie.mean() < 1e-3
+    same = got.view(np.int32) == want.view(np.int32)
+    assert same[~near_tie].all(), f"{int((~same & ~near_tie).sum())} results not correctly rounded"
+    # silu(+0) * 1 = +0 and silu(-0) * 1 = -0: the bit comparison above covered both signs
+    assert want[-10] == 0 and not np.signbit(want[-10]) and np.signbit(want[-9])
+
+
 def test_fused_gate_is_first_half():
     """silu(gate) * up with gate = columns [0, K), up = columns [K, 2K)."""
     K = 128

@@ -400,7 +400,7 @@ def test_ue8m0_bit_algorithm_equals_exact_ceiling():
     # random fp32 patterns in [1e-10, 2^127]
     lo = np.float32(1e-10).view(np.uint32)
     hi = np.float32(2.0 ** 127).view(np.uint32)
-    a_rand = rng.integers(lo, hi, size=2_000_000, dtype=np.uint32).view(np.float32)
+    a_rand = rng.integers(lo, hi, size=10_000_000, dtype=np.uint32).view(np.float32)
     # a near 7 * 2^k, where a/448 sits next to a power of two
     k = np.arange(-30, 120, dtype=np.float64)
     base = (7.0 * np.exp2(k)).astype(np.float32)
